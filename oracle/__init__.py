@@ -1,0 +1,21 @@
+"""fp64 CPU oracle for the fused attention forward pass — TEST INFRASTRUCTURE ONLY.
+
+What it computes is the plain definition of scaled-dot-product attention with the
+FlexAttention variants, written out in numpy float64: materialise the scores, apply the
+score modification and the mask, run a two-pass softmax, multiply by V, and report the
+per-row log-sum-exp.  It is deliberately slow and shares no code, header, table or
+constant with the CUDA path under ``tiled_attention_14_b200/``; neither imports the
+other.  Only the test suite, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
+``--impl reference`` legs of ``bench.py`` may import it.  The product path never calls
+it and has no CPU fallback.
+
+Modules
+-------
+``attention``  the attention forward (scores, score_mod, mask, softmax, O, LSE).
+``e4m3``       the FP8 e4m3 code book, encoder and per-128-row block quantiser.
+``tile_map``   the block-sparse tile classification (EMPTY / PARTIAL / FULL), by brute force.
+
+Every function is pinned by the ``-m "not gpu"`` tests in ``tests/test_oracle_*.py``
+against closed forms, invariants, brute force on tiny inputs and library routines
+(torch's CPU fp64 SDPA, torch's e4m3 cast).  No function is left "parity unpinned".
+"""
