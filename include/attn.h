@@ -1,0 +1,193 @@
+/*
+ * attn.h — C-ABI of libattn.so: fused scaled-dot-product attention forward for
+ * NVIDIA B200 (sm_100a), with the FlexAttention variants and an FP8 e4m3 path.
+ *
+ * What the calls compute
+ * ----------------------
+ *   O = softmax(score_mod(scale * Q K^T) masked by mask_mod) V,  LSE = ln sum exp(...)
+ * tile by tile with an online (running max / running sum) softmax, so the S x S score
+ * matrix never reaches HBM.  Definition: page "FlashAttention 4: Γρηγορότερη και
+ * Αποδοτική σε Μνήμη Προσοχή για LLMs", sections "Εισαγωγή" (softmax of Q K^T times V)
+ * and "Γιατί οι πυρήνες προσοχής ..." (tiles staged on chip, only the running max and
+ * sum kept per query row).  Variants: page "PyTorch's FlexAttention mit
+ * FlashAttention-4 ist ein Game-Changer", intro (ALiBi, sliding window, document
+ * masking, soft-capping) and section "Leistung und Validierung" (causal).  Block
+ * sparsity: same page, section "Aktuelle Einschränkungen".  FP8 with block
+ * quantisation: page "FlashAttention-3: Rekordverdächtige Geschwindigkeit ...",
+ * section "Analyse".
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Tensors are caller-owned DEVICE memory, contiguous, layout [B, H, S, D] (row i of
+ *   (b, h) at element offset ((b*H + h)*S + i)*D).  The library never frees or keeps
+ *   them and writes only the output arguments.
+ * - Pointers must be 16-byte aligned.  D is 64 or 128.  B, H, Sq, Sk >= 1 and
+ *   Sq, Sk <= ATTN_MAX_SEQ.
+ * - Causal alignment is bottom-right: query row i sits at key position
+ *   i' = i + (Sk - Sq).  CAUSAL keeps j <= i'.  WINDOW (width W >= 1) keeps
+ *   i' - j < W together with CAUSAL, |i' - j| < W without it.  DOC keeps
+ *   doc_ids[b, i] == doc_ids[b, j] and needs Sq == Sk.  The bits may be combined.
+ * - score_mod order: t = scale * q.k; if softcap > 0: t = softcap * tanh(t / softcap);
+ *   if alibi_slopes: t += alibi_slopes[h] * (j - i').
+ * - A query row that sees no key gets O = 0 and LSE = -inf.  LSE is natural-log.
+ * - Argument errors are returned synchronously and nothing is launched.  Launch
+ *   failures return ATTN_ERR_CUDA.  Errors raised inside a kernel (a bounded wait
+ *   that ran out) are recorded in a per-device status word read by attn_get_status.
+ * - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy default
+ *   stream).  The device must be compute capability 10.0 (B200); anything else gets
+ *   ATTN_ERR_UNSUPPORTED.
+ */
+#ifndef ATTN_H_
+#define ATTN_H_
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ATTN_API __attribute__((visibility("default")))
+#else
+#define ATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID = -1,      /* bad argument; nothing launched */
+  ATTN_ERR_UNSUPPORTED = -2,  /* device is not sm_100 */
+  ATTN_ERR_CUDA = -3,         /* a CUDA runtime/driver call or launch failed */
+  ATTN_ERR_TIMEOUT = -4,      /* a kernel's bounded wait ran out (from attn_get_status) */
+  ATTN_ERR_NOMEM = -5         /* workspace allocation failed */
+} attn_status;
+
+enum {
+  ATTN_MASK_NONE = 0,
+  ATTN_MASK_CAUSAL = 1,
+  ATTN_MASK_WINDOW = 2,
+  ATTN_MASK_DOC = 4
+};
+
+/* Tile-map geometry and entry format (see attn_tile_map_build). */
+enum {
+  ATTN_MAP_BLOCK_Q = 256,     /* query rows per map block: two 128-row query tiles */
+  ATTN_MAP_TILE_K = 128,      /* key columns per key tile */
+  ATTN_TILE_EMPTY = 0,
+  ATTN_TILE_PARTIAL = 1,
+  ATTN_TILE_FULL = 2
+};
+#define ATTN_MAP_ENTRY(kt, c0, c1) ((uint32_t)(kt) | ((uint32_t)(c0) << 24) | ((uint32_t)(c1) << 26))
+
+#define ATTN_MAX_SEQ (1 << 20)
+
+/*
+ * attn_fwd — BF16 attention forward.
+ *   q        bf16 [B,H,Sq,D]   (device, read)
+ *   k, v     bf16 [B,H,Sk,D]   (device, read)
+ *   o        bf16 [B,H,Sq,D]   (device, written)
+ *   lse      fp32 [B,H,Sq]     (device, written; natural log)
+ *   scale    finite, > 0 (usually 1/sqrt(D))
+ *   mask_kind  OR of ATTN_MASK_* bits
+ *   window   W >= 1, used iff the WINDOW bit is set
+ *   softcap  <= 0 turns soft-capping off; otherwise finite
+ *   alibi_slopes  device fp32 [H], or NULL for no ALiBi
+ *   doc_ids  device int32 [B,Sk], required iff the DOC bit is set (then Sq == Sk)
+ * With the DOC bit the call builds a tile map in a stream-ordered workspace
+ * (cudaMallocAsync / cudaFreeAsync on `stream`) and then runs the attention kernel;
+ * fully masked tiles are skipped.  CAUSAL and WINDOW tile ranges are computed in the
+ * kernel and need no workspace.  Accumulation is fp32; P is rounded to bf16 for P.V.
+ */
+ATTN_API int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+             int B, int H, int Sq, int Sk, int D, float scale,
+             int mask_kind, int window, float softcap,
+             const float* alibi_slopes, const int* doc_ids, void* stream);
+
+/*
+ * attn_tile_map_build — classify every (256-row query block, 128-column key tile) pair
+ * as EMPTY, PARTIAL or FULL under the mask and list the non-empty key tiles.
+ *   counts   device int32 [B, ceil(Sq/256)]               (written)
+ *   entries  device uint32 [B, ceil(Sq/256), ceil(Sk/128)] (written; only the first
+ *            counts[b,qb] entries of each row are meaningful)
+ * Entry = ATTN_MAP_ENTRY(kt, class of query tile 0, class of query tile 1), listed in
+ * increasing kt; a key tile is listed iff one of the two classes is not EMPTY.  EMPTY
+ * means no visible pair among valid rows (i < Sq) and keys (j < Sk); FULL means all
+ * 128 keys of the tile are valid and visible to every valid row; PARTIAL otherwise.
+ * The classification is exact (every pair is tested).  Mask arguments as attn_fwd;
+ * doc_ids may be NULL unless the DOC bit is set.
+ */
+ATTN_API int attn_tile_map_build(int* counts, uint32_t* entries, int B, int Sq, int Sk,
+                        int mask_kind, int window, const int* doc_ids, void* stream);
+
+/*
+ * attn_fwd_with_map — attn_fwd driven by a caller-supplied tile map (same format as
+ * attn_tile_map_build writes; same for every head).  The kernel visits exactly the
+ * listed key tiles, applies the element mask on PARTIAL tiles and trusts FULL tiles
+ * to need none.  A map that lists every key tile as PARTIAL computes the same result
+ * as skipping (fully masked tiles add exact zeros).  Other arguments as attn_fwd.
+ */
+ATTN_API int attn_fwd_with_map(const void* q, const void* k, const void* v, void* o, float* lse,
+                      int B, int H, int Sq, int Sk, int D, float scale,
+                      int mask_kind, int window, float softcap,
+                      const float* alibi_slopes, const int* doc_ids,
+                      const int* counts, const uint32_t* entries, void* stream);
+
+/*
+ * attn_quantize_e4m3 — per-block FP8 quantiser (FP8 with block quantisation: page
+ * "FlashAttention-3 ...", section "Analyse").  For each (b, h, block of 128 rows):
+ * a = max|x|; scales[b,h,blk] = a/448; xq = cvt.rn.satfinite.e4m3(x * (448/a)), both
+ * divisions correctly rounded fp32.  A block of zeros stores scale 1.
+ *   x       device fp32 [B,H,S,D]            (read)
+ *   xq      device e4m3 bytes [B,H,S,D]      (written)
+ *   scales  device fp32 [B,H,ceil(S/128)]    (written)
+ * D must be a multiple of 16 and at most 256.
+ */
+ATTN_API int attn_quantize_e4m3(const float* x, void* xq, float* scales, int B, int H, int S, int D,
+                       void* stream);
+
+/*
+ * attn_fwd_fp8 — attention forward on e4m3 Q, K, V with per-128-row fp32 block scales
+ * (as attn_quantize_e4m3 writes).  Scores use sQ*sK folded into the logit scale; P is
+ * quantised to e4m3 before P.V with the V block scale folded in as sV[kt]/max_kt(sV);
+ * the output is multiplied back by max_kt(sV).  Row sums use the unquantised P.
+ *   q8, k8, v8   device e4m3 [B,H,S,D]; q_scale/k_scale/v_scale device fp32
+ *   [B,H,ceil(S/128)]; o bf16 [B,H,Sq,D]; lse fp32 [B,H,Sq].
+ * Other arguments as attn_fwd (D = 128 only).
+ */
+ATTN_API int attn_fwd_fp8(const void* q8, const void* k8, const void* v8,
+                 const float* q_scale, const float* k_scale, const float* v_scale,
+                 void* o, float* lse,
+                 int B, int H, int Sq, int Sk, int D, float scale,
+                 int mask_kind, int window, float softcap,
+                 const float* alibi_slopes, const int* doc_ids, void* stream);
+
+/*
+ * attn_get_status — synchronises `stream`, then returns and clears the current device's
+ * status word: ATTN_OK, or ATTN_ERR_TIMEOUT if a kernel's bounded wait ran out since the
+ * last call (that kernel abandoned its work item and left its outputs undefined), or
+ * ATTN_ERR_CUDA if the synchronisation itself failed.
+ */
+ATTN_API int attn_get_status(void* stream);
+
+/* attn_strerror — static description of a status code (never NULL). */
+ATTN_API const char* attn_strerror(int code);
+
+/*
+ * attn_shutdown — releases host-side caches and returns the current device's pooled
+ * stream-ordered workspace memory to the system.  Safe to call more than once.
+ */
+ATTN_API void attn_shutdown(void);
+
+/*
+ * attn_debug_set_fault — test hook for the bounded waits.  A nonzero value makes the
+ * next attention launches skip one producer signal inside the kernel, so that the
+ * consumer's bounded wait runs out (about `timeout_ms` milliseconds) and the kernel
+ * records ATTN_ERR_TIMEOUT and returns.  0 restores normal operation.  Never set it in
+ * production.
+ */
+ATTN_API void attn_debug_set_fault(int skip_signal, int timeout_ms);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_H_ */

@@ -1,0 +1,74 @@
+"""Host-side checks of the C-ABI that need no GPU: the library loads, exports every symbol
+include/attn.h declares, and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from tiled_attention_14_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "attn.h")).read()
+    return re.findall(r"ATTN_API\s+[\w\s\*]+?\b(attn_\w+)\s*\(", src)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = _lib.load()
+    names = _declared()
+    assert set(names) == set(_lib.SIGNATURES), (names, sorted(_lib.SIGNATURES))
+    for n in names:
+        assert getattr(lib, n) is not None
+
+
+def test_strerror_is_static_text():
+    for code in (0, -1, -2, -3, -4, -5, 99):
+        assert isinstance(_lib.strerror(code), str) and _lib.strerror(code)
+
+
+A = 4096  # a fake, 16-byte aligned "device" address: argument checks fail before any use
+
+
+def _fwd(**kw):
+    args = dict(q=A, k=A, v=A, o=A, lse=A, B=1, H=1, Sq=128, Sk=128, D=128, scale=0.1, mask=0,
+                window=0, softcap=0.0, alibi=None, doc=None)
+    args.update(kw)
+    lib = _lib.load()
+    return lib.attn_fwd(args["q"], args["k"], args["v"], args["o"], args["lse"], args["B"], args["H"],
+                        args["Sq"], args["Sk"], args["D"], args["scale"], args["mask"], args["window"],
+                        args["softcap"], args["alibi"], args["doc"], None)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(q=None), dict(o=None), dict(lse=None), dict(k=A + 8), dict(D=96), dict(D=256), dict(Sq=0),
+    dict(Sk=-1), dict(B=0), dict(H=0), dict(scale=float("nan")), dict(scale=0.0), dict(scale=-1.0),
+    dict(scale=float("inf")), dict(mask=8), dict(mask=2, window=0), dict(mask=4),
+    dict(mask=4, doc=A, Sk=256), dict(softcap=float("inf")), dict(Sq=(1 << 20) + 1),
+    dict(alibi=A + 4), dict(doc=A + 4, mask=4)])
+def test_bad_arguments_rejected(kw):
+    assert _fwd(**kw) == _lib.ATTN_ERR_INVALID
+
+
+def test_bad_arguments_other_entry_points():
+    lib = _lib.load()
+    assert lib.attn_quantize_e4m3(A, A, A, 1, 1, 128, 96 + 8, None) == _lib.ATTN_ERR_INVALID
+    assert lib.attn_quantize_e4m3(None, A, A, 1, 1, 128, 64, None) == _lib.ATTN_ERR_INVALID
+    assert lib.attn_tile_map_build(None, A, 1, 128, 128, 0, 0, None, None) == _lib.ATTN_ERR_INVALID
+    assert lib.attn_tile_map_build(A, A, 1, 128, 256, 4, 0, A, None) == _lib.ATTN_ERR_INVALID
+    args = [A, A, A, A, A, 1, 1, 128, 128, 128, 0.1, 0, 0, 0.0, None, None]
+    assert lib.attn_fwd_with_map(*args, None, A, None) == _lib.ATTN_ERR_INVALID
+    fp8 = [A, A, A, A, A, A, A, A, 1, 1, 128, 128, 64, 0.1, 0, 0, 0.0, None, None, None]
+    assert lib.attn_fwd_fp8(*fp8) == _lib.ATTN_ERR_INVALID          # D = 64 unsupported for FP8
+    fp8[3] = None
+    fp8[12] = 128
+    assert lib.attn_fwd_fp8(*fp8) == _lib.ATTN_ERR_INVALID          # missing scales
+
+
+def test_wrapper_raises_on_missing_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(_lib, "_lib", None)
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "nope.so"))
+    with pytest.raises(RuntimeError):
+        _lib.load()

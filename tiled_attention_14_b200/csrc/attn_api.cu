@@ -1,0 +1,318 @@
+// attn_api.cu — host side of libattn.so: argument checks, TMA tensor-map encoding, kernel
+// selection and launch, the stream-ordered workspace, the device status word.
+//
+// The C-ABI is declared (with its contract) in include/attn.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "attn.h"
+#include "attn_fwd_kernel.cuh"
+#include "quant_kernel.cuh"
+#include "tile_map_kernel.cuh"
+
+namespace {
+
+using attn::FwdParams;
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool init = false;
+  bool supported = false;
+  int sms = 0;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::atomic<int> g_fault_skip{0};
+std::atomic<int> g_timeout_ms{1000};
+
+int current_device(int* dev) {
+  if (cudaGetDevice(dev) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (*dev < 0 || *dev >= kMaxDevices) return ATTN_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceInfo& d = g_dev[*dev];
+  if (!d.init) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, *dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, *dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, *dev) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    d.supported = (major == 10 && minor == 0);
+    d.sms = sms;
+    d.init = true;
+  }
+  if (!d.supported) return ATTN_ERR_UNSUPPORTED;
+  if (g_encode == nullptr) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr)
+      return ATTN_ERR_CUDA;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  return ATTN_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Checks shared by the attention entry points (host only; nothing is launched on failure).
+int check_common(const void* q, const void* k, const void* v, const void* o, const void* lse,
+                 int B, int H, int Sq, int Sk, int D, float scale, int mask_kind, int window,
+                 float softcap, const float* alibi, const int* doc_ids) {
+  if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return ATTN_ERR_INVALID;
+  if (alibi && !aligned16(alibi)) return ATTN_ERR_INVALID;
+  if (doc_ids && !aligned16(doc_ids)) return ATTN_ERR_INVALID;
+  if (D != 64 && D != 128) return ATTN_ERR_INVALID;
+  if (B <= 0 || H <= 0 || Sq <= 0 || Sk <= 0) return ATTN_ERR_INVALID;
+  if (Sq > ATTN_MAX_SEQ || Sk > ATTN_MAX_SEQ) return ATTN_ERR_INVALID;
+  if (static_cast<long long>(B) * H > (1LL << 24)) return ATTN_ERR_INVALID;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID;
+  if (mask_kind & ~(ATTN_MASK_CAUSAL | ATTN_MASK_WINDOW | ATTN_MASK_DOC)) return ATTN_ERR_INVALID;
+  if ((mask_kind & ATTN_MASK_WINDOW) && window <= 0) return ATTN_ERR_INVALID;
+  if ((mask_kind & ATTN_MASK_DOC) && (doc_ids == nullptr || Sq != Sk)) return ATTN_ERR_INVALID;
+  if (!std::isfinite(softcap)) return ATTN_ERR_INVALID;
+  return ATTN_OK;
+}
+
+int encode_map(CUtensorMap* map, const void* ptr, bool fp8, int BH, int S, int D) {
+  const int eb = fp8 ? 1 : 2;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(S), static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * eb, static_cast<cuuint64_t>(S) * D * eb};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / eb), 128u, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  const CUresult r = g_encode(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                              const_cast<void*>(ptr), dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <int D, bool FP8, bool SOFTCAP, bool ALIBI>
+int launch_fwd_t(int dev, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                 const FwdParams& p, cudaStream_t stream) {
+  using C = attn::Cfg<D, FP8>;
+  auto kern = attn::attn_fwd_kernel<D, FP8, SOFTCAP, ALIBI>;
+  static bool attr_set[kMaxDevices] = {};
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    attr_set[dev] = true;
+  }
+  const long long grid = static_cast<long long>(p.B) * p.H * p.nqb;
+  kern<<<static_cast<unsigned>(grid), attn::kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <int D, bool FP8>
+int launch_fwd_d(int dev, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                 const FwdParams& p, bool softcap, bool alibi, cudaStream_t s) {
+  if (softcap) {
+    return alibi ? launch_fwd_t<D, FP8, true, true>(dev, tq, tk, tv, p, s)
+                 : launch_fwd_t<D, FP8, true, false>(dev, tq, tk, tv, p, s);
+  }
+  return alibi ? launch_fwd_t<D, FP8, false, true>(dev, tq, tk, tv, p, s)
+               : launch_fwd_t<D, FP8, false, false>(dev, tq, tk, tv, p, s);
+}
+
+// Fills the parameter block shared by the BF16 and FP8 paths.
+FwdParams make_params(void* o, float* lse, int B, int H, int Sq, int Sk, float scale, int mask_kind,
+                      int window, float softcap, const float* alibi, const int* doc_ids) {
+  FwdParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.B = B;
+  p.H = H;
+  p.Sq = Sq;
+  p.Sk = Sk;
+  p.nqb = (Sq + 255) / 256;
+  p.nkt = (Sk + 127) / 128;
+  p.mask_kind = mask_kind;
+  // A window at least Sq + Sk wide removes nothing; clamping keeps the index math in int32.
+  const long long wmax = static_cast<long long>(Sq) + Sk;
+  p.window = (mask_kind & ATTN_MASK_WINDOW) ? static_cast<int>(window < wmax ? window : wmax) : 0;
+  const double log2e = 1.4426950408889634;
+  p.scale_log2 = static_cast<float>(static_cast<double>(scale) * log2e);
+  if (softcap > 0.f) {
+    p.sc_in = static_cast<float>(static_cast<double>(scale) / softcap);
+    p.sc_out = static_cast<float>(static_cast<double>(softcap) * log2e);
+  }
+  p.alibi = alibi;
+  p.doc = (mask_kind & ATTN_MASK_DOC) ? doc_ids : nullptr;
+  p.fault_skip = g_fault_skip.load();
+  p.timeout_ns = static_cast<unsigned long long>(g_timeout_ms.load()) * 1000000ull;
+  return p;
+}
+
+int launch_tile_map(int* counts, uint32_t* entries, int B, int Sq, int Sk, int mask_kind, int window,
+                    const int* doc_ids, cudaStream_t stream) {
+  const int nqb = (Sq + 255) / 256, nkt = (Sk + 127) / 128;
+  const long long wmax = static_cast<long long>(Sq) + Sk;
+  const int w = (mask_kind & ATTN_MASK_WINDOW) ? static_cast<int>(window < wmax ? window : wmax) : 0;
+  dim3 grid(nqb, B);
+  attn::tile_map_kernel<<<grid, attn::kMapThreads, 0, stream>>>(counts, entries, Sq, Sk, mask_kind, w,
+                                                                 (mask_kind & ATTN_MASK_DOC) ? doc_ids : nullptr,
+                                                                 nqb, nkt);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+size_t ws_bytes_for_map(int B, int Sq, int Sk) {
+  const size_t nc = static_cast<size_t>(B) * ((Sq + 255) / 256);
+  return ((nc * sizeof(int) + 15) & ~size_t(15)) + nc * ((Sk + 127) / 128) * sizeof(uint32_t);
+}
+
+// Shared body of attn_fwd / attn_fwd_with_map / attn_fwd_fp8.
+int run_fwd(bool fp8, const void* q, const void* k, const void* v, const float* qs, const float* ks,
+            const float* vs, void* o, float* lse, int B, int H, int Sq, int Sk, int D, float scale,
+            int mask_kind, int window, float softcap, const float* alibi, const int* doc_ids,
+            const int* counts, const uint32_t* entries, cudaStream_t stream) {
+  int rc = check_common(q, k, v, o, lse, B, H, Sq, Sk, D, scale, mask_kind, window, softcap, alibi, doc_ids);
+  if (rc != ATTN_OK) return rc;
+  if (fp8 && (D != 128 || !qs || !ks || !vs)) return ATTN_ERR_INVALID;
+  if ((counts == nullptr) != (entries == nullptr)) return ATTN_ERR_INVALID;
+  int dev = 0;
+  if ((rc = current_device(&dev)) != ATTN_OK) return rc;
+
+  FwdParams p = make_params(o, lse, B, H, Sq, Sk, scale, mask_kind, window, softcap, alibi, doc_ids);
+  if (fp8) {
+    p.q_scale = qs;
+    p.k_scale = ks;
+    p.v_scale = vs;
+    p.nsb_q = (Sq + 127) / 128;
+    p.nsb_k = (Sk + 127) / 128;
+  }
+  CUtensorMap tq, tk, tv;
+  if (encode_map(&tq, q, fp8, B * H, Sq, D) != ATTN_OK || encode_map(&tk, k, fp8, B * H, Sk, D) != ATTN_OK ||
+      encode_map(&tv, v, fp8, B * H, Sk, D) != ATTN_OK)
+    return ATTN_ERR_CUDA;
+
+  void* ws = nullptr;
+  if (counts == nullptr && (mask_kind & ATTN_MASK_DOC)) {
+    // Document masks need the tile map: a stream-ordered workspace for this call.
+    const size_t nc = static_cast<size_t>(B) * p.nqb;
+    if (cudaMallocAsync(&ws, ws_bytes_for_map(B, Sq, Sk), stream) != cudaSuccess) return ATTN_ERR_NOMEM;
+    int* c = static_cast<int*>(ws);
+    uint32_t* e = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + ((nc * sizeof(int) + 15) & ~size_t(15)));
+    rc = launch_tile_map(c, e, B, Sq, Sk, mask_kind, window, doc_ids, stream);
+    if (rc != ATTN_OK) {
+      cudaFreeAsync(ws, stream);
+      return rc;
+    }
+    counts = c;
+    entries = e;
+  }
+  p.map_counts = counts;
+  p.map_entries = entries;
+  const bool sc = softcap > 0.f, al = alibi != nullptr;
+  if (fp8) rc = launch_fwd_d<128, true>(dev, tq, tk, tv, p, sc, al, stream);
+  else if (D == 128) rc = launch_fwd_d<128, false>(dev, tq, tk, tv, p, sc, al, stream);
+  else rc = launch_fwd_d<64, false>(dev, tq, tk, tv, p, sc, al, stream);
+  if (ws) cudaFreeAsync(ws, stream);
+  return rc;
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Sq, int Sk,
+             int D, float scale, int mask_kind, int window, float softcap, const float* alibi_slopes,
+             const int* doc_ids, void* stream) {
+  return run_fwd(false, q, k, v, nullptr, nullptr, nullptr, o, lse, B, H, Sq, Sk, D, scale, mask_kind, window,
+                 softcap, alibi_slopes, doc_ids, nullptr, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+int attn_fwd_with_map(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Sq,
+                      int Sk, int D, float scale, int mask_kind, int window, float softcap,
+                      const float* alibi_slopes, const int* doc_ids, const int* counts, const uint32_t* entries,
+                      void* stream) {
+  if (!counts || !entries) return ATTN_ERR_INVALID;
+  return run_fwd(false, q, k, v, nullptr, nullptr, nullptr, o, lse, B, H, Sq, Sk, D, scale, mask_kind, window,
+                 softcap, alibi_slopes, doc_ids, counts, entries, static_cast<cudaStream_t>(stream));
+}
+
+int attn_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_scale, const float* k_scale,
+                 const float* v_scale, void* o, float* lse, int B, int H, int Sq, int Sk, int D, float scale,
+                 int mask_kind, int window, float softcap, const float* alibi_slopes, const int* doc_ids,
+                 void* stream) {
+  if (!q_scale || !k_scale || !v_scale) return ATTN_ERR_INVALID;
+  if (!aligned16(q_scale) || !aligned16(k_scale) || !aligned16(v_scale)) return ATTN_ERR_INVALID;
+  return run_fwd(true, q8, k8, v8, q_scale, k_scale, v_scale, o, lse, B, H, Sq, Sk, D, scale, mask_kind, window,
+                 softcap, alibi_slopes, doc_ids, nullptr, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+int attn_tile_map_build(int* counts, uint32_t* entries, int B, int Sq, int Sk, int mask_kind, int window,
+                        const int* doc_ids, void* stream) {
+  if (!counts || !entries) return ATTN_ERR_INVALID;
+  if (!aligned16(counts) || !aligned16(entries)) return ATTN_ERR_INVALID;
+  if (B <= 0 || Sq <= 0 || Sk <= 0 || Sq > ATTN_MAX_SEQ || Sk > ATTN_MAX_SEQ) return ATTN_ERR_INVALID;
+  if (B > 65535) return ATTN_ERR_INVALID;
+  if (mask_kind & ~(ATTN_MASK_CAUSAL | ATTN_MASK_WINDOW | ATTN_MASK_DOC)) return ATTN_ERR_INVALID;
+  if ((mask_kind & ATTN_MASK_WINDOW) && window <= 0) return ATTN_ERR_INVALID;
+  if ((mask_kind & ATTN_MASK_DOC) && (doc_ids == nullptr || Sq != Sk)) return ATTN_ERR_INVALID;
+  int dev = 0;
+  const int rc = current_device(&dev);
+  if (rc != ATTN_OK) return rc;
+  return launch_tile_map(counts, entries, B, Sq, Sk, mask_kind, window, doc_ids, static_cast<cudaStream_t>(stream));
+}
+
+int attn_quantize_e4m3(const float* x, void* xq, float* scales, int B, int H, int S, int D, void* stream) {
+  if (!x || !xq || !scales) return ATTN_ERR_INVALID;
+  if (!aligned16(x) || !aligned16(xq) || !aligned16(scales)) return ATTN_ERR_INVALID;
+  if (B <= 0 || H <= 0 || S <= 0 || D <= 0 || D % 16 != 0 || D > 256 || S > ATTN_MAX_SEQ) return ATTN_ERR_INVALID;
+  int dev = 0;
+  const int rc = current_device(&dev);
+  if (rc != ATTN_OK) return rc;
+  const int nsb = (S + 127) / 128;
+  const long long grid = static_cast<long long>(B) * H * nsb;
+  if (grid > 0x7fffffffLL) return ATTN_ERR_INVALID;
+  attn::quant_e4m3_kernel<<<static_cast<unsigned>(grid), attn::kQuantThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+      x, static_cast<uint8_t*>(xq), scales, S, D, nsb);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+int attn_get_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, attn::g_attn_status, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(attn::g_attn_status, &zero, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+  return v;
+}
+
+const char* attn_strerror(int code) {
+  switch (code) {
+    case ATTN_OK: return "ok";
+    case ATTN_ERR_INVALID: return "invalid argument";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported device (needs compute capability 10.0, B200)";
+    case ATTN_ERR_CUDA: return "CUDA error";
+    case ATTN_ERR_TIMEOUT: return "a bounded wait inside a kernel ran out";
+    case ATTN_ERR_NOMEM: return "workspace allocation failed";
+    default: return "unknown status";
+  }
+}
+
+void attn_shutdown(void) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return;
+  cudaMemPool_t pool;
+  if (cudaDeviceGetDefaultMemPool(&pool, dev) == cudaSuccess) cudaMemPoolTrimTo(pool, 0);
+}
+
+void attn_debug_set_fault(int skip_signal, int timeout_ms) {
+  g_fault_skip.store(skip_signal ? 1 : 0);
+  g_timeout_ms.store(timeout_ms > 0 ? timeout_ms : 1000);
+}
+
+}  // extern "C"
