@@ -1,0 +1,51 @@
+"""Host logic of bench.py (CPU only): exact FLOP counts against the oracle's brute-force
+visible-pair count, and the reference (oracle) arm's JSON line."""
+import json
+import os
+import subprocess
+import sys
+
+import numpy as np
+import pytest
+
+import bench
+from attn_workloads import MASK_CAUSAL, MASK_DOC, MASK_NONE, MASK_WINDOW, Workload, doc_ids_from_lengths, doc_lengths
+from oracle.attention import visible_pair_count
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.mark.parametrize("Sq,Sk,mask,W", [(300, 300, MASK_NONE, 0), (300, 300, MASK_CAUSAL, 0),
+                                          (200, 520, MASK_CAUSAL, 0), (520, 200, MASK_CAUSAL, 0),
+                                          (700, 700, MASK_CAUSAL | MASK_WINDOW, 128),
+                                          (700, 650, MASK_WINDOW, 77)])
+def test_visible_pairs_match_oracle(Sq, Sk, mask, W):
+    w = Workload("t", 2, 3, Sq, Sk, 64, mask, window=W)
+    assert bench.visible_pairs(w) == 6 * visible_pair_count(Sq, Sk, mask, W)
+
+
+@pytest.mark.parametrize("mask", [MASK_DOC, MASK_DOC | MASK_CAUSAL])
+def test_visible_pairs_documents(mask):
+    w = Workload("d", 2, 2, 8192, 8192, 128, mask, doc=True)
+    ref = sum(visible_pair_count(8192, 8192, mask, 0, doc_ids_from_lengths(doc_lengths(8192, b)))
+              for b in range(2)) * 2
+    assert bench.visible_pairs(w) == ref
+
+
+def test_benchmark_flop_counts():
+    assert bench.algorithmic_flops(bench.WORKLOADS["causal"]) == 4 * 128 * 64 * (4096 * 4097 // 2)
+    assert bench.algorithmic_flops(bench.WORKLOADS["long"]) == 4 * 128 * 32 * 32768 ** 2
+    # the kernel's 256x128 tiles cover a little more than the exact causal half
+    w = bench.WORKLOADS["causal"]
+    assert bench.tile_count_flops(w) > bench.algorithmic_flops(w)
+
+
+def test_reference_arm_prints_one_line():
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--workload", "tiny", "--steps", "1", "--warmup", "3"],
+                         capture_output=True, text=True, timeout=300, check=True).stdout
+    lines = [l for l in out.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "TFLOP/s" and d["value"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0

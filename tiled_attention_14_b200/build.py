@@ -7,6 +7,7 @@ The shared library is written next to this file, so that it travels with the sou
 from __future__ import annotations
 
 import os
+import re
 import shutil
 import subprocess
 import sys
@@ -47,13 +48,44 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
            "-shared", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
            "-I", INCLUDE, "-I", CSRC, "--expt-relaxed-constexpr",
            "-o", tmp] + [os.path.join(CSRC, s) for s in SOURCES] + list(extra or [])
+    cmd += ["-Xptxas", "-v"]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
-    subprocess.run(cmd, check=True)
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    if res.returncode != 0:
+        sys.stderr.write(res.stdout + res.stderr)
+        raise RuntimeError("nvcc failed")
+    check_registers(res.stderr)
+    if verbose:
+        sys.stderr.write(res.stderr)
     os.replace(tmp, LIB)
     return LIB
 
 
+# Registers per thread the attention kernels must be compiled to: the kernel's setmaxnreg
+# split (softmax warpgroups up, producer/MMA warpgroup down) adds up to exactly this many
+# per thread at launch, so any other count is a build error.
+LAUNCH_REGS = 168
+
+
+def check_registers(ptxas_log: str) -> None:
+    entry = None
+    seen = 0
+    for line in ptxas_log.splitlines():
+        m = re.search(r"Compiling entry function '([^']+)'", line)
+        if m:
+            entry = m.group(1)
+            continue
+        m = re.search(r"Used (\d+) registers", line)
+        if m and entry and "attn_fwd_kernel" in entry:
+            n = int(m.group(1))
+            if n != LAUNCH_REGS:
+                raise RuntimeError(f"{entry}: ptxas assigned {n} registers, the register split needs {LAUNCH_REGS}")
+            seen += 1
+            entry = None
+    if seen == 0:
+        raise RuntimeError("no attention kernel found in the ptxas report")
+
+
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose=True,
-          extra=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else None)
+    build(force="--force" in sys.argv, verbose="--ptxas-v" in sys.argv)

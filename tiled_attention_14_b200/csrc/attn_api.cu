@@ -76,7 +76,7 @@ int check_common(const void* q, const void* k, const void* v, const void* o, con
   if (D != 64 && D != 128) return ATTN_ERR_INVALID;
   if (B <= 0 || H <= 0 || Sq <= 0 || Sk <= 0) return ATTN_ERR_INVALID;
   if (Sq > ATTN_MAX_SEQ || Sk > ATTN_MAX_SEQ) return ATTN_ERR_INVALID;
-  if (static_cast<long long>(B) * H > (1LL << 24)) return ATTN_ERR_INVALID;
+  if (static_cast<long long>(B) * H * ((Sq + 255) / 256) > 0x7fffffffLL) return ATTN_ERR_INVALID;
   if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID;
   if (mask_kind & ~(ATTN_MASK_CAUSAL | ATTN_MASK_WINDOW | ATTN_MASK_DOC)) return ATTN_ERR_INVALID;
   if ((mask_kind & ATTN_MASK_WINDOW) && window <= 0) return ATTN_ERR_INVALID;
@@ -109,7 +109,9 @@ int launch_fwd_t(int dev, const CUtensorMap& tq, const CUtensorMap& tk, const CU
       return ATTN_ERR_CUDA;
     attr_set[dev] = true;
   }
-  const long long grid = static_cast<long long>(p.B) * p.H * p.nqb;
+  // Persistent grid: one CTA per SM (the kernel holds all 512 TMEM columns and most of
+  // shared memory, so only one CTA fits on an SM anyway), never more CTAs than work items.
+  const int grid = p.num_items < g_dev[dev].sms ? p.num_items : g_dev[dev].sms;
   kern<<<static_cast<unsigned>(grid), attn::kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
@@ -150,6 +152,10 @@ FwdParams make_params(void* o, float* lse, int B, int H, int Sq, int Sk, float s
   }
   p.alibi = alibi;
   p.doc = (mask_kind & ATTN_MASK_DOC) ? doc_ids : nullptr;
+  const long long items = static_cast<long long>(B) * H * p.nqb;
+  p.num_items = static_cast<int>(items);
+  // Causal without a window: query blocks differ a lot in length -> longest first.
+  p.lpt_qb_major = ((mask_kind & ATTN_MASK_CAUSAL) && !(mask_kind & (ATTN_MASK_WINDOW | ATTN_MASK_DOC))) ? 1 : 0;
   p.fault_skip = g_fault_skip.load();
   p.timeout_ns = static_cast<unsigned long long>(g_timeout_ms.load()) * 1000000ull;
   return p;

@@ -42,13 +42,32 @@
 
 namespace attn {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;          // three warpgroups
+// Register split (setmaxnreg): the kernel is launched with kLaunchRegs per thread
+// (384 x 168 = 64512 of the SM's 65536); the producer/MMA warpgroup gives registers back
+// and the two softmax warpgroups take them: 256 x 200 + 128 x 104 = 64512.  The build
+// checks that ptxas assigned exactly kLaunchRegs, otherwise an increase could never be met.
+constexpr int kLaunchRegs = 168;
+constexpr int kSoftmaxRegs = 200;
+constexpr int kControlRegs = 104;
+static_assert(256 * kSoftmaxRegs + 128 * kControlRegs == kThreads * kLaunchRegs, "register split");
 constexpr int kLoadWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr float kTau = 8.0f;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kNegInf = -__builtin_huge_valf();
+
+// Software exp2 (FMA pipes) takes one element pair in kSwExpEvery (0: all on MUFU).  Measured on
+// B200: with the packed-f32x2 softmax the exponentials are not MUFU-bound, so it is off.
+constexpr int kSwExpEvery = 0;
+constexpr int kSwDiv = kSwExpEvery > 0 ? kSwExpEvery : 1;
+// Coefficients of 2^f on [-1/2, 1/2] (near-minimax in relative error, fitted by
+// tiled_attention_14_b200/fit_exp2_poly.py; max relative error 7.5e-5 in float32).
+constexpr float kE0 = 0.9999280571937561f;
+constexpr float kE1 = 0.6932609677314758f;
+constexpr float kE2 = 0.2426111400127411f;
+constexpr float kE3 = 0.0551716685295105f;
 
 // Device status word (one per device that loads the library).
 __device__ int g_attn_status;
@@ -70,6 +89,8 @@ struct FwdParams {
   const float* k_scale;
   const float* v_scale;
   int nsb_q, nsb_k;
+  int num_items;           // B * H * nqb work items
+  int lpt_qb_major;        // 1: order work by query block first (causal: longest first)
   int fault_skip;          // test hook: group 1 skips its first P-ready signal
   unsigned long long timeout_ns;
 };
@@ -89,8 +110,8 @@ struct Cfg {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = 2 * TILE_BYTES;
   static constexpr int OFF_BAR = OFF_KV + NS * TILE_BYTES;
-  // barriers: q_full[2], kv_full[NS], kv_empty[NS], s_full[2], p_full[2], o_done[2], drain
-  static constexpr int NBAR = 2 + 2 * NS + 2 + 2 + 2 + 1;
+  // barriers: q_full[2], kv_full[NS], kv_empty[NS], s_full[2], p_full[2], o_done[2], drain, q_empty
+  static constexpr int NBAR = 2 + 2 * NS + 2 + 2 + 2 + 1 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;    // tmem base (4 B), abort flag (4 B)
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1024-byte alignment
   static constexpr uint32_t TMEM_COLS = 512;
@@ -98,6 +119,50 @@ struct Cfg {
   static constexpr uint32_t IDESC_QK = make_idesc(FP8 ? 0u : 1u, 128, 128, false);
   static constexpr uint32_t IDESC_PV = make_idesc(FP8 ? 0u : 1u, 128, D, true);
 };
+
+// ---------------------------------------------------------------------------------------
+// arithmetic helpers
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ float fmax3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Packed fp32 pair arithmetic (f32x2, sm_100): one instruction for two lanes of work,
+// rounding identical to the scalar forms.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+// 2^x on the FMA and integer pipes (software exp2, page "FlashAttention 4 ...", section
+// "Αποκορύφωση Λογισμικού μέσω Πυρήνων CUDA"): Cody-Waite split x = j + f with j the nearest
+// integer (added to 1.5*2^23 so that rounding leaves j in the low mantissa bits), a cubic
+// for 2^f, and j added straight into the exponent field.  x is clamped to >= -125 so the
+// result stays a normal float; callers that need exact zeros for -inf select them.
+__device__ __forceinline__ float exp2_fma(float x) {
+  x = fmaxf(x, -125.f);
+  const float r = x + 12582912.f;
+  const float j = r - 12582912.f;
+  const float f = x - j;
+  const float q = fmaf(fmaf(fmaf(kE3, f, kE2), f, kE1), f, kE0);
+  return __int_as_float(__float_as_int(q) + (__float_as_int(r) << 23));
+}
 
 // ---------------------------------------------------------------------------------------
 // bounded waiting
@@ -158,10 +223,19 @@ __device__ __forceinline__ int lo_key(const FwdParams& p, int ip) {  // first vi
   return (p.mask_kind & 2) ? ip - p.window + 1 : 0;
 }
 
-__device__ __forceinline__ Item make_item(const FwdParams& p, int item) {
+// Work item at position w of the schedule.  Causal masks (without a window) give the
+// 256-row query blocks very different lengths, so they are ordered longest first across
+// all heads; otherwise the order is head-major (the K/V of one head stay hot in L2).
+__device__ __forceinline__ Item make_item(const FwdParams& p, int w) {
   Item it;
-  it.bh = item / p.nqb;
-  it.qb = p.nqb - 1 - item % p.nqb;   // longest first within a head (causal)
+  const int BH = p.B * p.H;
+  if (p.lpt_qb_major) {
+    it.qb = p.nqb - 1 - w / BH;
+    it.bh = w % BH;
+  } else {
+    it.bh = w / p.nqb;
+    it.qb = p.nqb - 1 - w % p.nqb;
+  }
   it.b = it.bh / p.H;
   it.h = it.bh % p.H;
   it.entries = nullptr;
@@ -186,6 +260,12 @@ __device__ __forceinline__ Item make_item(const FwdParams& p, int item) {
   return it;
 }
 
+// Static persistent schedule: CTA b takes positions r*G + b (r even) or r*G + G-1-b (r odd),
+// r = 0, 1, ...  With the longest-first order this snake keeps the per-CTA totals even.
+__device__ __forceinline__ int sched_pos(int r, int b, int G) {
+  return r * G + ((r & 1) ? (G - 1 - b) : b);
+}
+
 __device__ __forceinline__ int tile_kt(const Item& it, int i) {
   return it.entries ? static_cast<int>(__ldg(it.entries + i) & 0xFFFFFFu) : it.kt_lo + i;
 }
@@ -208,8 +288,160 @@ __device__ __forceinline__ int tile_class(const FwdParams& p, const Item& it, in
   return full ? 2 : 1;
 }
 
+// One KV tile of one query tile's online softmax (every thread owns one query row): reads
+// the S row from TMEM, applies score_mod and the mask, updates the running max / sum with
+// the rescale threshold, writes P over S in TMEM, and rescales O when the max moved.
+template <int D, bool FP8, bool SOFTCAP, bool ALIBI>
+__device__ __forceinline__ void softmax_tile(const FwdParams& p, const Item& it, int kt, int cls, uint32_t tS,
+                                             uint32_t tO, int ip, int jlo_row, int jhi_row, bool has_doc,
+                                             int doc_row, float slope_l2, float sq_scale, float v_norm,
+                                             float& m_run, float& l_run) {
+  using C = Cfg<D, FP8>;
+      uint32_t s[128];
+      tmem_ld_x128_wait(tS, s);
+      float sc = p.scale_log2;     // raw score -> log2 units
+      float sc_in = p.sc_in;       // raw score -> tanh argument
+      float pv_factor = 1.f;
+      if constexpr (FP8) {
+        const size_t kb = static_cast<size_t>(it.bh) * p.nsb_k + kt;
+        const float sqk = sq_scale * __ldg(p.k_scale + kb);
+        sc *= sqk;
+        sc_in *= sqk;
+        pv_factor = __ldg(p.v_scale + kb) / v_norm;
+      }
+      const int c0 = kt * 128;
+      // ---- score_mod (log2 units) and mask; row maximum as a shallow max3 tree
+      constexpr bool kPlain = !SOFTCAP && !ALIBI;
+      float alibi_base = 0.f;
+      if constexpr (ALIBI) alibi_base = slope_l2 * static_cast<float>(c0 - ip);
+      auto modify = [&](float t, int c) -> float {
+        if constexpr (!kPlain) {
+          if constexpr (SOFTCAP) {
+            // tanh(x) = sign(x) (1 - 2 / (e^{2|x|} + 1)): absolute error ~1e-7
+            const float x = t * sc_in;
+            const float e = ex2_approx(fabsf(x) * (2.f * kLog2e));
+            t = copysignf(1.f - 2.f * rcp_approx(e + 1.f), x) * p.sc_out;
+          } else {
+            t *= sc;
+          }
+          if constexpr (ALIBI) t = fmaf(slope_l2, static_cast<float>(c), t + alibi_base);
+        }
+        return t;
+      };
+      float mxa[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) mxa[u] = kNegInf;
+      const bool masked = (cls == 1);
+      if (masked) {
+        const int clo = jlo_row - c0, chi = jhi_row - c0;
+        const int* dk = p.doc + static_cast<size_t>(it.b) * p.Sk + c0;
+        const int nvalid = p.Sk - c0;
+#pragma unroll
+        for (int c = 0; c < 128; c += 2) {
+          float t0 = modify(__uint_as_float(s[c]), c);
+          float t1 = modify(__uint_as_float(s[c + 1]), c + 1);
+          bool v0 = (c >= clo) && (c <= chi);
+          bool v1 = (c + 1 >= clo) && (c + 1 <= chi);
+          if (has_doc) {
+            v0 = v0 && (c < nvalid) && (__ldg(dk + min(c, nvalid - 1)) == doc_row);
+            v1 = v1 && (c + 1 < nvalid) && (__ldg(dk + min(c + 1, nvalid - 1)) == doc_row);
+          }
+          t0 = v0 ? t0 : kNegInf;
+          t1 = v1 ? t1 : kNegInf;
+          s[c] = __float_as_uint(t0);
+          s[c + 1] = __float_as_uint(t1);
+          mxa[(c >> 1) & 7] = fmax3f(mxa[(c >> 1) & 7], t0, t1);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 128; c += 2) {
+          const float t0 = modify(__uint_as_float(s[c]), c);
+          const float t1 = modify(__uint_as_float(s[c + 1]), c + 1);
+          if constexpr (!kPlain) {
+            s[c] = __float_as_uint(t0);
+            s[c + 1] = __float_as_uint(t1);
+          }
+          mxa[(c >> 1) & 7] = fmax3f(mxa[(c >> 1) & 7], t0, t1);
+        }
+      }
+      float mx = fmax3f(fmax3f(mxa[0], mxa[1], mxa[2]), fmax3f(mxa[3], mxa[4], mxa[5]),
+                        fmaxf(mxa[6], mxa[7]));
+      // In the plain case the scores are still raw: scale the maximum (scale > 0).
+      if constexpr (kPlain) mx = mx * sc;
+      // ---- online softmax with the rescale threshold
+      bool rescale = false;
+      float alpha = 1.f;
+      if (mx > m_run + kTau) {
+        if (m_run != kNegInf) {
+          alpha = ex2_approx(m_run - mx);
+          rescale = true;
+          l_run *= alpha;
+        }
+        m_run = mx;
+      }
+      const float msub = (m_run == kNegInf) ? 0.f : m_run;
+      // ---- exponentials, packed two per register (f32x2 FMA / ADD), P to TMEM in two halves
+      const float2 sc2 = make_float2(sc, sc);
+      const float2 nm2 = make_float2(-msub, -msub);
+      // 2^a: with kSwExpEvery > 0, one pair in kSwExpEvery goes to the FMA pipes (software
+      // exp2); the split depends on the column only, so FULL and PARTIAL tiles agree bit for bit.
+      auto pexp = [&](float a, int c) -> float {
+        if (kSwExpEvery > 0 && (c >> 1) % kSwDiv == kSwDiv - 1) {
+          const float e = exp2_fma(a);
+          return masked ? (a == kNegInf ? 0.f : e) : e;
+        }
+        return ex2_approx(a);
+      };
+      auto arg2 = [&](int c) -> float2 {
+        const float2 v = make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+        if constexpr (kPlain) return ffma2(v, sc2, nm2);
+        else return fadd2(v, nm2);
+      };
+      float2 ls[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) ls[u] = make_float2(0.f, 0.f);
+      uint32_t pk[C::P_COLS];
+      if constexpr (!FP8) {
+#pragma unroll
+        for (int c2 = 0; c2 < 64; ++c2) {
+          const float2 a = arg2(2 * c2);
+          const float2 pp = make_float2(pexp(a.x, 2 * c2), pexp(a.y, 2 * c2 + 1));
+          ls[c2 & 3] = fadd2(ls[c2 & 3], pp);
+          pk[c2] = pack_bf16x2(pp.x, pp.y);
+          if (c2 == 31) tmem_st_x32_nowait<0>(tS, pk);
+        }
+        tmem_st_x32_wait<32>(tS + 32, pk);
+      } else {
+#pragma unroll
+        for (int c4 = 0; c4 < 32; ++c4) {
+          const float2 a = arg2(4 * c4), b = arg2(4 * c4 + 2);
+          const float2 p01 = make_float2(pexp(a.x, 4 * c4), pexp(a.y, 4 * c4 + 1));
+          const float2 p23 = make_float2(pexp(b.x, 4 * c4 + 2), pexp(b.y, 4 * c4 + 3));
+          ls[c4 & 3] = fadd2(ls[c4 & 3], fadd2(p01, p23));
+          pk[c4] = pack_e4m3x2(p01.x * pv_factor, p01.y * pv_factor) |
+                   (pack_e4m3x2(p23.x * pv_factor, p23.y * pv_factor) << 16);
+          if (c4 == 15) tmem_st_x16_nowait<0>(tS, pk);
+        }
+        tmem_st_x16_wait<16>(tS + 16, pk);
+      }
+      const float2 l2 = fadd2(fadd2(ls[0], ls[1]), fadd2(ls[2], ls[3]));
+      l_run += l2.x + l2.y;
+      // ---- rescale O when the maximum moved by more than TAU (PV_g(i-1) is complete:
+      //      its commit preceded the one that signalled S_g(i)).
+      if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+        for (int ch = 0; ch < D / 32; ++ch) {
+          uint32_t o[32];
+          tmem_ld_x32_wait(tO + ch * 32, o);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+          tmem_st_x32_wait<0>(tO + ch * 32, o);
+        }
+      }
+}
+
 // ---------------------------------------------------------------------------------------
-// the kernel
+// the kernel (persistent: one CTA per SM walks its share of the work items)
 // ---------------------------------------------------------------------------------------
 template <int D, bool FP8, bool SOFTCAP, bool ALIBI>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -222,13 +454,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   uint8_t* sptr = smem_raw + (sbase - raw);
   auto BAR = [&](int i) -> uint32_t { return sbase + C::OFF_BAR + 8 * i; };
   const int B_QFULL = 0, B_KVFULL = 2, B_KVEMPTY = 2 + C::NS, B_SFULL = 2 + 2 * C::NS,
-            B_PFULL = B_SFULL + 2, B_ODONE = B_PFULL + 2, B_DRAIN = B_ODONE + 2;
+            B_PFULL = B_SFULL + 2, B_ODONE = B_PFULL + 2, B_DRAIN = B_ODONE + 2, B_QEMPTY = B_DRAIN + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sptr + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sptr + C::OFF_MISC + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const Item it = make_item(p, blockIdx.x);
+  const int G = gridDim.x;
+  const int cta = blockIdx.x;
   const unsigned long long tmo = p.timeout_ns;
 
   if (threadIdx.x == 0) {
@@ -244,6 +477,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       mbar_init(BAR(B_ODONE + g), 1);
     }
     mbar_init(BAR(B_DRAIN), 1);
+    mbar_init(BAR(B_QEMPTY), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -260,43 +494,53 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_holder;
-
+  if (warp >= 8) {
+    setmaxnreg_dec<kControlRegs>();
   if (warp == kLoadWarp) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       const uint64_t pol_kv = policy_evict_last();
       const uint64_t pol_q = policy_evict_first();
-      for (int g = 0; g < 2; ++g) {
-        mbar_expect_tx(BAR(B_QFULL + g), C::TILE_BYTES);
-        for (int pn = 0; pn < C::NPANEL; ++pn)
-          tma_load_3d(sbase + C::OFF_Q + g * C::TILE_BYTES + pn * C::PANEL_BYTES, &tm_q,
-                      BAR(B_QFULL + g), pn * C::PANEL_COLS, it.qb * 256 + 128 * g, it.bh, pol_q);
-      }
-      int issued = 0;  // loads issued into the ring
-      for (int i = 0; i < it.n; ++i) {
-        const int kt = tile_kt(it, i);
-        bool ok = true;
-        for (int kv = 0; kv < 2 && ok; ++kv) {
-          const int idx = 2 * i + kv;
-          const int slot = idx % C::NS;
-          const uint32_t par = ((idx / C::NS) & 1) ^ 1;
-          if (!wait_bounded(BAR(B_KVEMPTY + slot), par, abort_flag, tmo)) {
-            ok = false;
-            break;
-          }
-          mbar_expect_tx(BAR(B_KVFULL + slot), C::TILE_BYTES);
-          const CUtensorMap* tm = kv ? &tm_v : &tm_k;
+      uint32_t lidx = 0;     // ring loads issued (K and V alternate)
+      uint32_t qcount = 0;   // Q tile pairs issued
+      bool ok = true;
+      for (int r = 0; ok; ++r) {
+        const int w = sched_pos(r, cta, G);
+        if (w >= p.num_items) break;
+        const Item it = make_item(p, w);
+        if (it.n == 0) continue;
+        // Q smem is free once every S MMA of the previous item has completed.
+        if (qcount > 0 && !wait_bounded(BAR(B_QEMPTY), (qcount - 1) & 1, abort_flag, tmo)) break;
+        for (int g = 0; g < 2; ++g) {
+          mbar_expect_tx(BAR(B_QFULL + g), C::TILE_BYTES);
           for (int pn = 0; pn < C::NPANEL; ++pn)
-            tma_load_3d(sbase + C::OFF_KV + slot * C::TILE_BYTES + pn * C::PANEL_BYTES, tm,
-                        BAR(B_KVFULL + slot), pn * C::PANEL_COLS, kt * 128, it.bh, pol_kv);
-          ++issued;
+            tma_load_3d(sbase + C::OFF_Q + g * C::TILE_BYTES + pn * C::PANEL_BYTES, &tm_q,
+                        BAR(B_QFULL + g), pn * C::PANEL_COLS, it.qb * 256 + 128 * g, it.bh, pol_q);
         }
-        if (!ok) break;
+        ++qcount;
+        for (int i = 0; i < it.n && ok; ++i) {
+          const int kt = tile_kt(it, i);
+          for (int kv = 0; kv < 2; ++kv) {
+            const uint32_t slot = lidx % C::NS;
+            if (!wait_bounded(BAR(B_KVEMPTY + slot), ((lidx / C::NS) & 1) ^ 1, abort_flag, tmo)) {
+              ok = false;
+              break;
+            }
+            mbar_expect_tx(BAR(B_KVFULL + slot), C::TILE_BYTES);
+            const CUtensorMap* tm = kv ? &tm_v : &tm_k;
+            for (int pn = 0; pn < C::NPANEL; ++pn)
+              tma_load_3d(sbase + C::OFF_KV + slot * C::TILE_BYTES + pn * C::PANEL_BYTES, tm,
+                          BAR(B_KVFULL + slot), pn * C::PANEL_COLS, kt * 128, it.bh, pol_kv);
+            ++lidx;
+          }
+        }
       }
       // Drain: every copy issued by this thread has landed before the CTA may exit.
-      drain_bounded(BAR(B_QFULL + 0), 0, tmo);
-      drain_bounded(BAR(B_QFULL + 1), 0, tmo);
-      for (int idx = max(0, issued - C::NS); idx < issued; ++idx)
+      if (qcount > 0) {
+        drain_bounded(BAR(B_QFULL + 0), (qcount - 1) & 1, tmo);
+        drain_bounded(BAR(B_QFULL + 1), (qcount - 1) & 1, tmo);
+      }
+      for (uint32_t idx = (lidx > C::NS ? lidx - C::NS : 0); idx < lidx; ++idx)
         drain_bounded(BAR(B_KVFULL + idx % C::NS), (idx / C::NS) & 1, tmo);
     }
   } else if (warp == kMmaWarp) {
@@ -304,274 +548,187 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (lane == 0) {
       const uint32_t tS[2] = {tbase + C::T_S0, tbase + C::T_S1};
       const uint32_t tO[2] = {tbase + C::T_O0, tbase + C::T_O1};
-      const uint32_t sQ[2] = {sbase + C::OFF_Q, sbase + C::OFF_Q + C::TILE_BYTES};
-      auto qk = [&](int g, int kslot) {
-        const uint32_t kbase = sbase + C::OFF_KV + kslot * C::TILE_BYTES;
+      // Descriptors of the first tiles; a byte offset b inside the shared window is added as
+      // b >> 4 to the start-address field (all addresses stay below 256 KB, so no carry).
+      const uint64_t dq = make_sdesc_sw128(sbase + C::OFF_Q, 16, 1024);
+      const uint64_t dk = make_sdesc_sw128(sbase + C::OFF_KV, 16, 1024);
+      const uint64_t dv = make_sdesc_sw128(sbase + C::OFF_KV, C::PANEL_BYTES, 1024);
+      auto qk = [&](int g, uint32_t kslot) {
+        const uint64_t a0 = dq + ((g * C::TILE_BYTES) >> 4);
+        const uint64_t b0 = dk + ((kslot * C::TILE_BYTES) >> 4);
 #pragma unroll
         for (int kk = 0; kk < C::QK_STEPS; ++kk) {
           const int col = kk * C::KSTEP;
-          const uint32_t off = (col / C::PANEL_COLS) * C::PANEL_BYTES + (col % C::PANEL_COLS) * C::EB;
-          const uint64_t ad = make_sdesc_sw128(sQ[g] + off, 16, 1024);
-          const uint64_t bd = make_sdesc_sw128(kbase + off, 16, 1024);
-          if constexpr (FP8) mma_f8_ss(tS[g], ad, bd, C::IDESC_QK, kk > 0);
-          else mma_f16_ss(tS[g], ad, bd, C::IDESC_QK, kk > 0);
+          const uint32_t off = ((col / C::PANEL_COLS) * C::PANEL_BYTES + (col % C::PANEL_COLS) * C::EB) >> 4;
+          if constexpr (FP8) mma_f8_ss(tS[g], a0 + off, b0 + off, C::IDESC_QK, kk > 0);
+          else mma_f16_ss(tS[g], a0 + off, b0 + off, C::IDESC_QK, kk > 0);
         }
       };
-      auto pv = [&](int g, int vslot, bool acc) {
-        const uint32_t vbase = sbase + C::OFF_KV + vslot * C::TILE_BYTES;
+      auto pv = [&](int g, uint32_t vslot, bool acc) {
+        const uint64_t b0 = dv + ((vslot * C::TILE_BYTES) >> 4);
 #pragma unroll
         for (int kk = 0; kk < C::PV_STEPS; ++kk) {
-          const uint64_t bd = make_sdesc_sw128(vbase + kk * C::KSTEP * 128, C::PANEL_BYTES, 1024);
+          const uint64_t bd = b0 + ((kk * C::KSTEP * 128) >> 4);
           const uint32_t ta = tS[g] + kk * (C::KSTEP * C::EB / 4);
           if constexpr (FP8) mma_f8_ts(tO[g], ta, bd, C::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
           else mma_f16_ts(tO[g], ta, bd, C::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
         }
       };
-      bool ok = wait_bounded(BAR(B_QFULL + 0), 0, abort_flag, tmo) &&
-                wait_bounded(BAR(B_QFULL + 1), 0, abort_flag, tmo);
-      int prev_vslot = 0;
-      for (int i = 0; i < it.n && ok; ++i) {
-        const int kidx = 2 * i, vidx = 2 * i + 1;
-        const int kslot = kidx % C::NS, vslot = vidx % C::NS;
-        // S0(i) = Q0 K_i^T   (S0 holds P0(i-1) until PV0(i-1) has completed)
-        if (!wait_bounded(BAR(B_KVFULL + kslot), (kidx / C::NS) & 1, abort_flag, tmo)) break;
-        if (i > 0 && !wait_bounded(BAR(B_ODONE + 0), (i - 1) & 1, abort_flag, tmo)) break;
-        tc_fence_after();
-        qk(0, kslot);
-        mma_commit(BAR(B_SFULL + 0));
-        // O1 += P1(i-1) V_{i-1}
-        if (i > 0) {
-          if (!wait_bounded(BAR(B_PFULL + 1), (i - 1) & 1, abort_flag, tmo)) { ok = false; break; }
-          tc_fence_after();
-          pv(1, prev_vslot, i - 1 > 0);
-          mma_commit(BAR(B_ODONE + 1));
-          mma_commit(BAR(B_KVEMPTY + prev_vslot));
-          if (!wait_bounded(BAR(B_ODONE + 1), (i - 1) & 1, abort_flag, tmo)) { ok = false; break; }
-          tc_fence_after();
+      uint32_t cidx = 0;     // ring loads consumed
+      uint32_t tcount = 0;   // tiles processed (phase of s_full / p_full / o_done)
+      uint32_t qcount = 0;
+      bool ok = true;
+      for (int r = 0; ok; ++r) {
+        const int w = sched_pos(r, cta, G);
+        if (w >= p.num_items) break;
+        const Item it = make_item(p, w);
+        if (it.n == 0) continue;
+        if (!wait_bounded(BAR(B_QFULL + 0), qcount & 1, abort_flag, tmo) ||
+            !wait_bounded(BAR(B_QFULL + 1), qcount & 1, abort_flag, tmo)) {
+          ok = false;
+          break;
         }
-        // S1(i) = Q1 K_i^T
-        qk(1, kslot);
-        mma_commit(BAR(B_SFULL + 1));
-        mma_commit(BAR(B_KVEMPTY + kslot));
-        // O0 += P0(i) V_i
-        if (!wait_bounded(BAR(B_KVFULL + vslot), (vidx / C::NS) & 1, abort_flag, tmo)) break;
-        if (!wait_bounded(BAR(B_PFULL + 0), i & 1, abort_flag, tmo)) break;
-        tc_fence_after();
-        pv(0, vslot, i > 0);
-        mma_commit(BAR(B_ODONE + 0));
-        prev_vslot = vslot;
-      }
-      if (ok && it.n > 0 && !*abort_flag) {
+        uint32_t prev_vslot = 0;
+        for (int i = 0; i < it.n; ++i) {
+          const uint32_t t = tcount + i;
+          const uint32_t kidx = cidx + 2 * i, vidx = kidx + 1;
+          const uint32_t kslot = kidx % C::NS, vslot = vidx % C::NS;
+          // S0(i) = Q0 K_i^T.  It overwrites P0(i-1), which PV0(i-1) (issued earlier by this
+          // thread) reads: tcgen05.mma operations from one thread execute in issue order.
+          if (!wait_bounded(BAR(B_KVFULL + kslot), (kidx / C::NS) & 1, abort_flag, tmo)) { ok = false; break; }
+          tc_fence_after();
+          qk(0, kslot);
+          mma_commit(BAR(B_SFULL + 0));
+          // O1 += P1(i-1) V_{i-1}
+          if (i > 0) {
+            if (!wait_bounded(BAR(B_PFULL + 1), (t - 1) & 1, abort_flag, tmo)) { ok = false; break; }
+            tc_fence_after();
+            pv(1, prev_vslot, i - 1 > 0);
+            mma_commit(BAR(B_ODONE + 1));
+            mma_commit(BAR(B_KVEMPTY + prev_vslot));
+          }
+          // S1(i) = Q1 K_i^T
+          qk(1, kslot);
+          mma_commit(BAR(B_SFULL + 1));
+          mma_commit(BAR(B_KVEMPTY + kslot));
+          if (i == it.n - 1) mma_commit(BAR(B_QEMPTY));   // the last reads of Q for this item
+          // O0 += P0(i) V_i
+          if (!wait_bounded(BAR(B_KVFULL + vslot), (vidx / C::NS) & 1, abort_flag, tmo)) { ok = false; break; }
+          if (!wait_bounded(BAR(B_PFULL + 0), t & 1, abort_flag, tmo)) { ok = false; break; }
+          tc_fence_after();
+          pv(0, vslot, i > 0);
+          mma_commit(BAR(B_ODONE + 0));
+          prev_vslot = vslot;
+        }
+        if (!ok) break;
         // O1 += P1(n-1) V_{n-1}
-        if (wait_bounded(BAR(B_PFULL + 1), (it.n - 1) & 1, abort_flag, tmo)) {
-          tc_fence_after();
-          pv(1, prev_vslot, it.n - 1 > 0);
-          mma_commit(BAR(B_ODONE + 1));
-          mma_commit(BAR(B_KVEMPTY + prev_vslot));
-        }
+        const uint32_t tl = tcount + it.n - 1;
+        if (!wait_bounded(BAR(B_PFULL + 1), tl & 1, abort_flag, tmo)) { ok = false; break; }
+        tc_fence_after();
+        pv(1, prev_vslot, it.n - 1 > 0);
+        mma_commit(BAR(B_ODONE + 1));
+        mma_commit(BAR(B_KVEMPTY + prev_vslot));
+        cidx += 2 * it.n;
+        tcount += it.n;
+        ++qcount;
       }
       // Drain: all MMAs issued by this thread are complete before TMEM is freed.
       mma_commit(BAR(B_DRAIN));
       drain_bounded(BAR(B_DRAIN), 0, tmo);
     }
+  }
   } else {
+    setmaxnreg_inc<kSoftmaxRegs>();
     // ------------------------------------------------------------------ softmax groups
     const int g = warp >> 2;                       // query tile of this group
     const int rloc = (warp & 3) * 32 + lane;       // row within the query tile (= TMEM lane)
-    const int row = it.qb * 256 + 128 * g + rloc;  // query row
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tbase + (g ? C::T_S1 : C::T_S0) + lane_off;
     const uint32_t tO = tbase + (g ? C::T_O1 : C::T_O0) + lane_off;
-    const int ip = row + (p.Sk - p.Sq);            // bottom-right aligned position
-    const int jlo_row = lo_key(p, ip);
-    const int jhi_row = hi_key(p, ip);
     const bool has_doc = (p.mask_kind & 4) != 0;
-    const int doc_row = (has_doc && row < p.Sq) ? __ldg(p.doc + static_cast<size_t>(it.b) * p.Sk + row) : 0;
-    float slope_l2 = 0.f;
-    if constexpr (ALIBI) slope_l2 = __ldg(p.alibi + it.h) * kLog2e;
-    float sq_scale = 1.f, v_norm = 1.f;
-    if constexpr (FP8) {
-      const size_t qbase = static_cast<size_t>(it.bh) * p.nsb_q;
-      sq_scale = __ldg(p.q_scale + qbase + min(2 * it.qb + g, p.nsb_q - 1));
-      const size_t vbase = static_cast<size_t>(it.bh) * p.nsb_k;
-      float vm = 0.f;
-      for (int sb = 0; sb < p.nsb_k; ++sb) vm = fmaxf(vm, __ldg(p.v_scale + vbase + sb));
-      v_norm = vm > 0.f ? vm : 1.f;
-    }
-
-    float m_run = kNegInf;   // running maximum used for the exponentials (log2 units)
-    float l_run = 0.f;       // running row sum against m_run
+    uint32_t tcount = 0;
     bool ok = true;
-    for (int i = 0; i < it.n; ++i) {
-      const int kt = tile_kt(it, i);
-      const int cls = tile_class(p, it, i, g, kt);
-      if (!wait_bounded(BAR(B_SFULL + g), i & 1, abort_flag, tmo)) { ok = false; break; }
-      tc_fence_after();
-      if (cls == 0) {
-        // Fully masked for this query tile: P = 0, m and l unchanged.
-        uint32_t z[C::P_COLS];
-#pragma unroll
-        for (int c = 0; c < C::P_COLS; ++c) z[c] = 0u;
-        if constexpr (C::P_COLS == 64) tmem_st_x64_wait(tS, z);
-        else tmem_st_x32_wait(tS, z);
-      } else {
-        uint32_t s[128];
-        tmem_ld_x128_wait(tS, s);
-        float sc = p.scale_log2;     // raw score -> log2 units
-        float sc_in = p.sc_in;       // raw score -> tanh argument
-        float pv_factor = 1.f;
-        if constexpr (FP8) {
-          const size_t kb = static_cast<size_t>(it.bh) * p.nsb_k + kt;
-          const float sqk = sq_scale * __ldg(p.k_scale + kb);
-          sc *= sqk;
-          sc_in *= sqk;
-          pv_factor = __ldg(p.v_scale + kb) / v_norm;
-        }
-        const int c0 = kt * 128;
-        // ---- score_mod (log2 units) and mask; row maximum
-        float mx = kNegInf;
-        constexpr bool kPlain = !SOFTCAP && !ALIBI;
-        if (cls == 1) {
-          const int clo = jlo_row - c0, chi = jhi_row - c0;
-          const int* dk = p.doc + static_cast<size_t>(it.b) * p.Sk + c0;
-          const int nvalid = p.Sk - c0;
-#pragma unroll
-          for (int c = 0; c < 128; ++c) {
-            float t = __uint_as_float(s[c]);
-            if constexpr (!kPlain) {
-              if constexpr (SOFTCAP) {
-                const float x = t * sc_in;
-                const float e = ex2_approx(fabsf(x) * (2.f * kLog2e));
-                t = copysignf(1.f - 2.f * rcp_approx(e + 1.f), x) * p.sc_out;
-              } else {
-                t *= sc;
-              }
-              if constexpr (ALIBI) t = fmaf(slope_l2, static_cast<float>(c), t + slope_l2 * static_cast<float>(c0 - ip));
-            }
-            bool vis = (c >= clo) && (c <= chi);
-            if (has_doc) vis = vis && (c < nvalid) && (__ldg(dk + min(c, nvalid - 1)) == doc_row);
-            t = vis ? t : kNegInf;
-            s[c] = __float_as_uint(t);
-            mx = fmaxf(mx, t);
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < 128; ++c) {
-            float t = __uint_as_float(s[c]);
-            if constexpr (!kPlain) {
-              if constexpr (SOFTCAP) {
-                const float x = t * sc_in;
-                const float e = ex2_approx(fabsf(x) * (2.f * kLog2e));
-                t = copysignf(1.f - 2.f * rcp_approx(e + 1.f), x) * p.sc_out;
-              } else {
-                t *= sc;
-              }
-              if constexpr (ALIBI) t = fmaf(slope_l2, static_cast<float>(c), t + slope_l2 * static_cast<float>(c0 - ip));
-              s[c] = __float_as_uint(t);
-            }
-            mx = fmaxf(mx, t);
-          }
-        }
-        // In the plain case the scores are still raw: scale the maximum (scale > 0).
-        if constexpr (kPlain) mx = mx * sc;
-        // ---- online softmax with the rescale threshold
-        bool rescale = false;
-        float alpha = 1.f;
-        if (mx > m_run + kTau) {
-          if (m_run != kNegInf) {
-            alpha = ex2_approx(m_run - mx);
-            rescale = true;
-            l_run *= alpha;
-          }
-          m_run = mx;
-        }
-        const float msub = (m_run == kNegInf) ? 0.f : m_run;
-        float l0 = 0.f, l1 = 0.f;
-        uint32_t pk[C::P_COLS];
-        if constexpr (!FP8) {
-#pragma unroll
-          for (int c2 = 0; c2 < 64; ++c2) {
-            float a0, a1;
-            if constexpr (kPlain) {
-              a0 = fmaf(__uint_as_float(s[2 * c2]), sc, -msub);
-              a1 = fmaf(__uint_as_float(s[2 * c2 + 1]), sc, -msub);
-            } else {
-              a0 = __uint_as_float(s[2 * c2]) - msub;
-              a1 = __uint_as_float(s[2 * c2 + 1]) - msub;
-            }
-            const float p0 = ex2_approx(a0), p1 = ex2_approx(a1);
-            l0 += p0;
-            l1 += p1;
-            pk[c2] = pack_bf16x2(p0, p1);
-          }
-          tmem_st_x64_wait(tS, pk);
-        } else {
-#pragma unroll
-          for (int c4 = 0; c4 < 32; ++c4) {
-            float pp[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              float a;
-              if constexpr (kPlain) a = fmaf(__uint_as_float(s[4 * c4 + u]), sc, -msub);
-              else a = __uint_as_float(s[4 * c4 + u]) - msub;
-              pp[u] = ex2_approx(a);
-            }
-            l0 += pp[0] + pp[2];
-            l1 += pp[1] + pp[3];
-            pk[c4] = pack_e4m3x2(pp[0] * pv_factor, pp[1] * pv_factor) |
-                     (pack_e4m3x2(pp[2] * pv_factor, pp[3] * pv_factor) << 16);
-          }
-          tmem_st_x32_wait(tS, pk);
-        }
-        l_run += l0 + l1;
-        // ---- rescale O when the maximum moved by more than TAU (PV_g(i-1) is complete:
-        //      its commit preceded the one that signalled S_g(i)).
-        if (__any_sync(0xffffffffu, rescale)) {
-#pragma unroll
-          for (int ch = 0; ch < D / 32; ++ch) {
-            uint32_t o[32];
-            tmem_ld_x32_wait(tO + ch * 32, o);
-#pragma unroll
-            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-            tmem_st_x32_wait(tO + ch * 32, o);
-          }
-        }
+    for (int r = 0; ok; ++r) {
+      const int w = sched_pos(r, cta, G);
+      if (w >= p.num_items) break;
+      const Item it = make_item(p, w);
+      const int row = it.qb * 256 + 128 * g + rloc;  // query row
+      const int ip = row + (p.Sk - p.Sq);            // bottom-right aligned position
+      const int jlo_row = lo_key(p, ip);
+      const int jhi_row = hi_key(p, ip);
+      const int doc_row = (has_doc && row < p.Sq) ? __ldg(p.doc + static_cast<size_t>(it.b) * p.Sk + row) : 0;
+      float slope_l2 = 0.f;
+      if constexpr (ALIBI) slope_l2 = __ldg(p.alibi + it.h) * kLog2e;
+      float sq_scale = 1.f, v_norm = 1.f;
+      if constexpr (FP8) {
+        const size_t qbase = static_cast<size_t>(it.bh) * p.nsb_q;
+        sq_scale = __ldg(p.q_scale + qbase + min(2 * it.qb + g, p.nsb_q - 1));
+        const size_t vbase = static_cast<size_t>(it.bh) * p.nsb_k;
+        float vm = 0.f;
+        for (int sb = 0; sb < p.nsb_k; ++sb) vm = fmaxf(vm, __ldg(p.v_scale + vbase + sb));
+        v_norm = vm > 0.f ? vm : 1.f;
       }
-      tc_fence_before();
-      if (!(p.fault_skip && g == 1 && i == 0)) mbar_arrive(BAR(B_PFULL + g));
-    }
-    // ---- epilogue: O / l -> bf16, LSE
-    if (ok && !*abort_flag) {
-      bool have = true;
-      if (it.n > 0) have = wait_bounded(BAR(B_ODONE + g), (it.n - 1) & 1, abort_flag, tmo);
-      if (have) {
+
+      float m_run = kNegInf;   // running maximum used for the exponentials (log2 units)
+      float l_run = 0.f;       // running row sum against m_run
+      for (int i = 0; i < it.n; ++i) {
+        const uint32_t t = tcount + i;
+        const int kt = tile_kt(it, i);
+        const int cls = tile_class(p, it, i, g, kt);
+        if (!wait_bounded(BAR(B_SFULL + g), t & 1, abort_flag, tmo)) { ok = false; break; }
         tc_fence_after();
-        const float inv_l = (l_run > 0.f) ? (v_norm / l_run) : 0.f;
-        __nv_bfloat16* orow = p.o + (static_cast<size_t>(it.bh) * p.Sq + row) * D;
+        if (cls == 0) {
+          // Fully masked for this query tile: P = 0, m and l unchanged.
+          uint32_t z[C::P_COLS];
 #pragma unroll
-        for (int ch = 0; ch < D / 32; ++ch) {
-          uint32_t o[32];
-          if (it.n > 0) {
-            tmem_ld_x32_wait(tO + ch * 32, o);
-          } else {
-#pragma unroll
-            for (int c = 0; c < 32; ++c) o[c] = 0u;
-          }
-          uint32_t w[16];
-#pragma unroll
-          for (int c = 0; c < 16; ++c)
-            w[c] = pack_bf16x2(__uint_as_float(o[2 * c]) * inv_l, __uint_as_float(o[2 * c + 1]) * inv_l);
-          if (row < p.Sq) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
-#pragma unroll
-            for (int v = 0; v < 4; ++v) dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
-          }
+          for (int c = 0; c < C::P_COLS; ++c) z[c] = 0u;
+          if constexpr (C::P_COLS == 64) tmem_st_x64_wait<0>(tS, z);
+          else tmem_st_x32_wait<0>(tS, z);
+        } else {
+          softmax_tile<D, FP8, SOFTCAP, ALIBI>(p, it, kt, cls, tS, tO, ip, jlo_row, jhi_row, has_doc,
+                                               doc_row, slope_l2, sq_scale, v_norm, m_run, l_run);
         }
+        tc_fence_before();
+        if (!(p.fault_skip && g == 1 && t == 0)) mbar_arrive(BAR(B_PFULL + g));
+      }
+      if (!ok || *abort_flag) {
+        ok = false;
+        break;
+      }
+      // ---- epilogue: O / l -> bf16, LSE
+      if (it.n > 0) {
+        if (!wait_bounded(BAR(B_ODONE + g), (tcount + it.n - 1) & 1, abort_flag, tmo)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+      }
+      const float inv_l = (l_run > 0.f) ? (v_norm / l_run) : 0.f;
+      __nv_bfloat16* orow = p.o + (static_cast<size_t>(it.bh) * p.Sq + row) * D;
+#pragma unroll
+      for (int ch = 0; ch < D / 32; ++ch) {
+        uint32_t o[32];
+        if (it.n > 0) {
+          tmem_ld_x32_wait(tO + ch * 32, o);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = 0u;
+        }
+        uint32_t wv[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+          wv[c] = pack_bf16x2(__uint_as_float(o[2 * c]) * inv_l, __uint_as_float(o[2 * c + 1]) * inv_l);
         if (row < p.Sq) {
-          const float lse = (l_run > 0.f) ? (m_run + lg2_approx(l_run)) * kLn2 : kNegInf;
-          p.lse[static_cast<size_t>(it.bh) * p.Sq + row] = lse;
+          uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(wv[4 * v], wv[4 * v + 1], wv[4 * v + 2], wv[4 * v + 3]);
         }
       }
+      if (row < p.Sq) {
+        const float lse = (l_run > 0.f) ? (m_run + lg2_approx(l_run)) * kLn2 : kNegInf;
+        p.lse[static_cast<size_t>(it.bh) * p.Sq + row] = lse;
+      }
+      tcount += it.n;
     }
   }
 

@@ -163,6 +163,16 @@ __device__ __forceinline__ uint64_t make_sdesc_sw128(uint32_t addr, uint32_t lbo
   return d;
 }
 
+// Per-warpgroup register budget (all four warps of the warpgroup execute it).
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ---------------------------------------------------------------------------------------
 // MUFU approximations and conversions
 // ---------------------------------------------------------------------------------------
