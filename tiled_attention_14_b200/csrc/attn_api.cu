@@ -162,20 +162,25 @@ FwdParams make_params(void* o, float* lse, int B, int H, int Sq, int Sk, float s
 }
 
 int launch_tile_map(int* counts, uint32_t* entries, int B, int Sq, int Sk, int mask_kind, int window,
-                    const int* doc_ids, cudaStream_t stream) {
+                    const int* doc_ids, cudaStream_t stream, int* sorted_flags = nullptr) {
   const int nqb = (Sq + 255) / 256, nkt = (Sk + 127) / 128;
   const long long wmax = static_cast<long long>(Sq) + Sk;
   const int w = (mask_kind & ATTN_MASK_WINDOW) ? static_cast<int>(window < wmax ? window : wmax) : 0;
   dim3 grid(nqb, B);
   attn::tile_map_kernel<<<grid, attn::kMapThreads, 0, stream>>>(counts, entries, Sq, Sk, mask_kind, w,
                                                                  (mask_kind & ATTN_MASK_DOC) ? doc_ids : nullptr,
-                                                                 nqb, nkt);
+                                                                 nqb, nkt, sorted_flags);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
+// Workspace of the document path: counts [B*nqb] | entries [B*nqb*nkt] | sorted flags [B],
+// each part 16-byte aligned.
+size_t ws_counts_bytes(int B, int Sq) { return ((static_cast<size_t>(B) * ((Sq + 255) / 256) * sizeof(int) + 15) & ~size_t(15)); }
+size_t ws_entries_bytes(int B, int Sq, int Sk) {
+  return ((static_cast<size_t>(B) * ((Sq + 255) / 256) * ((Sk + 127) / 128) * sizeof(uint32_t) + 15) & ~size_t(15));
+}
 size_t ws_bytes_for_map(int B, int Sq, int Sk) {
-  const size_t nc = static_cast<size_t>(B) * ((Sq + 255) / 256);
-  return ((nc * sizeof(int) + 15) & ~size_t(15)) + nc * ((Sk + 127) / 128) * sizeof(uint32_t);
+  return ws_counts_bytes(B, Sq) + ws_entries_bytes(B, Sq, Sk) + static_cast<size_t>(B) * sizeof(int);
 }
 
 // Shared body of attn_fwd / attn_fwd_with_map / attn_fwd_fp8.
@@ -206,11 +211,12 @@ int run_fwd(bool fp8, const void* q, const void* k, const void* v, const float* 
   void* ws = nullptr;
   if (counts == nullptr && (mask_kind & ATTN_MASK_DOC)) {
     // Document masks need the tile map: a stream-ordered workspace for this call.
-    const size_t nc = static_cast<size_t>(B) * p.nqb;
     if (cudaMallocAsync(&ws, ws_bytes_for_map(B, Sq, Sk), stream) != cudaSuccess) return ATTN_ERR_NOMEM;
     int* c = static_cast<int*>(ws);
-    uint32_t* e = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + ((nc * sizeof(int) + 15) & ~size_t(15)));
-    rc = launch_tile_map(c, e, B, Sq, Sk, mask_kind, window, doc_ids, stream);
+    uint32_t* e = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + ws_counts_bytes(B, Sq));
+    int* sorted = reinterpret_cast<int*>(static_cast<char*>(ws) + ws_counts_bytes(B, Sq) + ws_entries_bytes(B, Sq, Sk));
+    rc = launch_tile_map(c, e, B, Sq, Sk, mask_kind, window, doc_ids, stream, sorted);
+    p.doc_sorted = sorted;
     if (rc != ATTN_OK) {
       cudaFreeAsync(ws, stream);
       return rc;

@@ -54,6 +54,7 @@ static_assert(256 * kSoftmaxRegs + 128 * kControlRegs == kThreads * kLaunchRegs,
 constexpr int kLoadWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr float kTau = 8.0f;
+constexpr int kPrefetchTiles = 3;      // K/V tiles warmed into L2 ahead of the smem ring
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kNegInf = -__builtin_huge_valf();
@@ -82,6 +83,7 @@ struct FwdParams {
   float sc_in, sc_out;     // soft-capping: x = s * sc_in, t = tanh(x) * sc_out (log2 units)
   const float* alibi;      // [H] slopes or nullptr
   const int* doc;          // [B, Sk] or nullptr
+  const int* doc_sorted;   // [B]: 1 if doc[b, :] is non-decreasing (from the tile-map build), or nullptr
   const int* map_counts;   // [B, nqb] or nullptr (analytic ranges)
   const uint32_t* map_entries;  // [B, nqb, nkt]
   // FP8 block scales [B, H, nsb] (nullptr for bf16)
@@ -110,8 +112,8 @@ struct Cfg {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = 2 * TILE_BYTES;
   static constexpr int OFF_BAR = OFF_KV + NS * TILE_BYTES;
-  // barriers: q_full[2], kv_full[NS], kv_empty[NS], s_full[2], p_full[2], o_done[2], drain, q_empty
-  static constexpr int NBAR = 2 + 2 * NS + 2 + 2 + 2 + 1 + 1;
+  // barriers: q_full[2], kv_full[NS], kv_empty[NS], s_full[2], p_full[2], o_done[2], drain, q_empty[2]
+  static constexpr int NBAR = 2 + 2 * NS + 2 + 2 + 2 + 1 + 2;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;    // tmem base (4 B), abort flag (4 B)
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1024-byte alignment
   static constexpr uint32_t TMEM_COLS = 512;
@@ -310,7 +312,8 @@ __device__ __forceinline__ void softmax_tile(const FwdParams& p, const Item& it,
         pv_factor = __ldg(p.v_scale + kb) / v_norm;
       }
       const int c0 = kt * 128;
-      // ---- score_mod (log2 units) and mask; row maximum as a shallow max3 tree
+      // ---- score_mod (log2 units) and mask; row maximum as a shallow max3 tree.  Each
+      //      variant is its own unrolled loop: no runtime branch inside the 128 columns.
       constexpr bool kPlain = !SOFTCAP && !ALIBI;
       float alibi_base = 0.f;
       if constexpr (ALIBI) alibi_base = slope_l2 * static_cast<float>(c0 - ip);
@@ -333,24 +336,35 @@ __device__ __forceinline__ void softmax_tile(const FwdParams& p, const Item& it,
       for (int u = 0; u < 8; ++u) mxa[u] = kNegInf;
       const bool masked = (cls == 1);
       if (masked) {
+        // visible columns of this row: clo <= c <= chi (causal / window / sorted documents),
+        // and, for unsorted document ids, doc[c] == doc of the row
         const int clo = jlo_row - c0, chi = jhi_row - c0;
-        const int* dk = p.doc + static_cast<size_t>(it.b) * p.Sk + c0;
-        const int nvalid = p.Sk - c0;
+        if (!has_doc) {
 #pragma unroll
-        for (int c = 0; c < 128; c += 2) {
-          float t0 = modify(__uint_as_float(s[c]), c);
-          float t1 = modify(__uint_as_float(s[c + 1]), c + 1);
-          bool v0 = (c >= clo) && (c <= chi);
-          bool v1 = (c + 1 >= clo) && (c + 1 <= chi);
-          if (has_doc) {
-            v0 = v0 && (c < nvalid) && (__ldg(dk + min(c, nvalid - 1)) == doc_row);
-            v1 = v1 && (c + 1 < nvalid) && (__ldg(dk + min(c + 1, nvalid - 1)) == doc_row);
+          for (int c = 0; c < 128; c += 2) {
+            float t0 = modify(__uint_as_float(s[c]), c);
+            float t1 = modify(__uint_as_float(s[c + 1]), c + 1);
+            t0 = (c >= clo && c <= chi) ? t0 : kNegInf;
+            t1 = (c + 1 >= clo && c + 1 <= chi) ? t1 : kNegInf;
+            s[c] = __float_as_uint(t0);
+            s[c + 1] = __float_as_uint(t1);
+            mxa[(c >> 1) & 7] = fmax3f(mxa[(c >> 1) & 7], t0, t1);
           }
-          t0 = v0 ? t0 : kNegInf;
-          t1 = v1 ? t1 : kNegInf;
-          s[c] = __float_as_uint(t0);
-          s[c + 1] = __float_as_uint(t1);
-          mxa[(c >> 1) & 7] = fmax3f(mxa[(c >> 1) & 7], t0, t1);
+        } else {
+          const int* dk = p.doc + static_cast<size_t>(it.b) * p.Sk + c0;
+          const int nvalid = p.Sk - c0;
+#pragma unroll
+          for (int c = 0; c < 128; c += 2) {
+            float t0 = modify(__uint_as_float(s[c]), c);
+            float t1 = modify(__uint_as_float(s[c + 1]), c + 1);
+            const bool v0 = c >= clo && c <= chi && c < nvalid && __ldg(dk + min(c, nvalid - 1)) == doc_row;
+            const bool v1 = c + 1 >= clo && c + 1 <= chi && c + 1 < nvalid && __ldg(dk + min(c + 1, nvalid - 1)) == doc_row;
+            t0 = v0 ? t0 : kNegInf;
+            t1 = v1 ? t1 : kNegInf;
+            s[c] = __float_as_uint(t0);
+            s[c + 1] = __float_as_uint(t1);
+            mxa[(c >> 1) & 7] = fmax3f(mxa[(c >> 1) & 7], t0, t1);
+          }
         }
       } else {
 #pragma unroll
@@ -477,7 +491,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       mbar_init(BAR(B_ODONE + g), 1);
     }
     mbar_init(BAR(B_DRAIN), 1);
-    mbar_init(BAR(B_QEMPTY), 1);
+    mbar_init(BAR(B_QEMPTY + 0), 1);
+    mbar_init(BAR(B_QEMPTY + 1), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -509,17 +524,44 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (w >= p.num_items) break;
         const Item it = make_item(p, w);
         if (it.n == 0) continue;
-        // Q smem is free once every S MMA of the previous item has completed.
-        if (qcount > 0 && !wait_bounded(BAR(B_QEMPTY), (qcount - 1) & 1, abort_flag, tmo)) break;
+        // Query tile g's smem is free once the previous item's last S_g MMA has completed.
         for (int g = 0; g < 2; ++g) {
+          if (qcount > 0 && !wait_bounded(BAR(B_QEMPTY + g), (qcount - 1) & 1, abort_flag, tmo)) {
+            ok = false;
+            break;
+          }
           mbar_expect_tx(BAR(B_QFULL + g), C::TILE_BYTES);
           for (int pn = 0; pn < C::NPANEL; ++pn)
             tma_load_3d(sbase + C::OFF_Q + g * C::TILE_BYTES + pn * C::PANEL_BYTES, &tm_q,
                         BAR(B_QFULL + g), pn * C::PANEL_COLS, it.qb * 256 + 128 * g, it.bh, pol_q);
         }
+        if (!ok) break;
         ++qcount;
+        // Warm L2 with the next item's query tiles and first key/value tiles.
+        for (int r2 = r + 1;; ++r2) {
+          const int w2 = sched_pos(r2, cta, G);
+          if (w2 >= p.num_items) break;
+          const Item nx = make_item(p, w2);
+          if (nx.n == 0) continue;
+          for (int pn = 0; pn < C::NPANEL; ++pn) {
+            tma_prefetch_l2_3d(&tm_q, pn * C::PANEL_COLS, nx.qb * 256, nx.bh);
+            tma_prefetch_l2_3d(&tm_q, pn * C::PANEL_COLS, nx.qb * 256 + 128, nx.bh);
+            for (int j = 0; j < min(nx.n, kPrefetchTiles); ++j) {
+              tma_prefetch_l2_3d(&tm_k, pn * C::PANEL_COLS, tile_kt(nx, j) * 128, nx.bh);
+              tma_prefetch_l2_3d(&tm_v, pn * C::PANEL_COLS, tile_kt(nx, j) * 128, nx.bh);
+            }
+          }
+          break;
+        }
         for (int i = 0; i < it.n && ok; ++i) {
           const int kt = tile_kt(it, i);
+          if (i + kPrefetchTiles < it.n) {
+            const int ktp = tile_kt(it, i + kPrefetchTiles);
+            for (int pn = 0; pn < C::NPANEL; ++pn) {
+              tma_prefetch_l2_3d(&tm_k, pn * C::PANEL_COLS, ktp * 128, it.bh);
+              tma_prefetch_l2_3d(&tm_v, pn * C::PANEL_COLS, ktp * 128, it.bh);
+            }
+          }
           for (int kv = 0; kv < 2; ++kv) {
             const uint32_t slot = lidx % C::NS;
             if (!wait_bounded(BAR(B_KVEMPTY + slot), ((lidx / C::NS) & 1) ^ 1, abort_flag, tmo)) {
@@ -599,6 +641,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           tc_fence_after();
           qk(0, kslot);
           mma_commit(BAR(B_SFULL + 0));
+          if (i == it.n - 1) mma_commit(BAR(B_QEMPTY + 0));   // last read of Q0 for this item
           // O1 += P1(i-1) V_{i-1}
           if (i > 0) {
             if (!wait_bounded(BAR(B_PFULL + 1), (t - 1) & 1, abort_flag, tmo)) { ok = false; break; }
@@ -611,7 +654,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           qk(1, kslot);
           mma_commit(BAR(B_SFULL + 1));
           mma_commit(BAR(B_KVEMPTY + kslot));
-          if (i == it.n - 1) mma_commit(BAR(B_QEMPTY));   // the last reads of Q for this item
+          if (i == it.n - 1) mma_commit(BAR(B_QEMPTY + 1));   // last read of Q1 for this item
           // O0 += P0(i) V_i
           if (!wait_bounded(BAR(B_KVFULL + vslot), (vidx / C::NS) & 1, abort_flag, tmo)) { ok = false; break; }
           if (!wait_bounded(BAR(B_PFULL + 0), t & 1, abort_flag, tmo)) { ok = false; break; }
@@ -654,9 +697,25 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const Item it = make_item(p, w);
       const int row = it.qb * 256 + 128 * g + rloc;  // query row
       const int ip = row + (p.Sk - p.Sq);            // bottom-right aligned position
-      const int jlo_row = lo_key(p, ip);
-      const int jhi_row = hi_key(p, ip);
+      int jlo_row = lo_key(p, ip);
+      int jhi_row = hi_key(p, ip);
       const int doc_row = (has_doc && row < p.Sq) ? __ldg(p.doc + static_cast<size_t>(it.b) * p.Sk + row) : 0;
+      bool doc_elem = has_doc;   // per-element document test needed on PARTIAL tiles
+      if (has_doc && p.doc_sorted != nullptr && __ldg(p.doc_sorted + it.b) != 0) {
+        // Non-decreasing ids: the row's document is one run, found by two binary searches,
+        // and the visible keys stay one interval.
+        if (row < p.Sq) {
+          const int* drow = p.doc + static_cast<size_t>(it.b) * p.Sk;
+          int lo = 0, hi = p.Sk;
+          while (lo < hi) { const int mid = (lo + hi) >> 1; if (__ldg(drow + mid) < doc_row) lo = mid + 1; else hi = mid; }
+          const int ds = lo;
+          hi = p.Sk;
+          while (lo < hi) { const int mid = (lo + hi) >> 1; if (__ldg(drow + mid) <= doc_row) lo = mid + 1; else hi = mid; }
+          jlo_row = max(jlo_row, ds);
+          jhi_row = min(jhi_row, lo - 1);
+        }
+        doc_elem = false;
+      }
       float slope_l2 = 0.f;
       if constexpr (ALIBI) slope_l2 = __ldg(p.alibi + it.h) * kLog2e;
       float sq_scale = 1.f, v_norm = 1.f;
@@ -685,7 +744,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           if constexpr (C::P_COLS == 64) tmem_st_x64_wait<0>(tS, z);
           else tmem_st_x32_wait<0>(tS, z);
         } else {
-          softmax_tile<D, FP8, SOFTCAP, ALIBI>(p, it, kt, cls, tS, tO, ip, jlo_row, jhi_row, has_doc,
+          softmax_tile<D, FP8, SOFTCAP, ALIBI>(p, it, kt, cls, tS, tO, ip, jlo_row, jhi_row, doc_elem,
                                                doc_row, slope_l2, sq_scale, v_norm, m_run, l_run);
         }
         tc_fence_before();

@@ -15,6 +15,8 @@
 //  * otherwise the kernel tests every (row, key) pair of the tile (exact, slower).
 // Per tile the rows' answers are reduced per query tile with warp votes and shared memory,
 // then the non-empty tiles are compacted in increasing order with a block prefix sum.
+// Optionally it records, per batch row, whether the document ids are non-decreasing (the
+// attention kernel then tests documents as key intervals instead of element by element).
 #pragma once
 #include <cstdint>
 
@@ -42,7 +44,8 @@ __device__ __forceinline__ int upper_bound_i32(const int* a, int n, int v) {
 
 __global__ void __launch_bounds__(kMapThreads)
 tile_map_kernel(int* __restrict__ counts, uint32_t* __restrict__ entries, int Sq, int Sk,
-                int mask_kind, int window, const int* __restrict__ doc, int nqb, int nkt) {
+                int mask_kind, int window, const int* __restrict__ doc, int nqb, int nkt,
+                int* __restrict__ sorted_flags) {
   __shared__ uint8_t w_any[8][kMapChunk];
   __shared__ uint8_t w_all[8][kMapChunk];
   __shared__ int kdoc[128];
@@ -68,6 +71,7 @@ tile_map_kernel(int* __restrict__ counts, uint32_t* __restrict__ entries, int Sq
     for (int j = t; j + 1 < Sk; j += kMapThreads)
       if (__ldg(drow + j) > __ldg(drow + j + 1)) sorted = false;
     sorted = __syncthreads_and(sorted);
+    if (sorted_flags != nullptr && qb == 0 && t == 0) sorted_flags[b] = sorted ? 1 : 0;
     if (valid) {
       mydoc = __ldg(drow + row);
       if (sorted) {
