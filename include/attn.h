@@ -103,6 +103,27 @@ ATTN_API int attn_fwd(const void* q, const void* k, const void* v, void* o, floa
              const float* alibi_slopes, const int* doc_ids, void* stream);
 
 /*
+ * attn_fwd_noalloc — attn_fwd that allocates no device memory.  (An addition of this
+ * library; the method itself has no counterpart for it.)
+ * Meant for callers that cannot allocate during a call: code inside a framework whose own
+ * caching allocator owns device memory, serving loops where an allocation or free could
+ * synchronise the device mid-request, and programs with a fixed memory budget.  The tile
+ * map of the DOC bit goes into a library-owned static device array of
+ * ATTN_NOALLOC_SCRATCH_BYTES (4 MiB) per device, held until the process exits; a map that
+ * needs more (bytes ~ 4*B*ceil(Sq/256)*ceil(Sk/128)) returns ATTN_ERR_INVALID, nothing
+ * launched.  Without the DOC bit no scratch is used at all.  The first call on a device
+ * looks up the array's device address (cudaGetSymbolAddress, with that device current),
+ * so make that first call before any stream capture.  All calls on one device share the
+ * array: calls whose kernels may overlap on the GPU race on it and must be ordered (one
+ * stream, or events).  Arguments, outputs and errors as attn_fwd (BF16, D = 64 or 128).
+ */
+#define ATTN_NOALLOC_SCRATCH_BYTES (4 << 20)
+ATTN_API int attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
+                              int B, int H, int Sq, int Sk, int D, float scale,
+                              int mask_kind, int window, float softcap,
+                              const float* alibi_slopes, const int* doc_ids, void* stream);
+
+/*
  * attn_tile_map_build — classify every (256-row query block, 128-column key tile) pair
  * as EMPTY, PARTIAL or FULL under the mask and list the non-empty key tiles.
  *   counts   device int32 [B, ceil(Sq/256)]               (written)

@@ -13,7 +13,7 @@ import torch
 from ._lib import (ATTN_ERR_TIMEOUT, ATTN_OK, MASK_CAUSAL, MASK_DOC, MASK_NONE, MASK_WINDOW,
                    AttnError, check, load)
 
-__all__ = ["attn_fwd", "attn_fwd_with_map", "attn_fwd_fp8", "attn_quantize_e4m3",
+__all__ = ["attn_fwd", "attn_fwd_noalloc", "attn_fwd_with_map", "attn_fwd_fp8", "attn_quantize_e4m3",
            "attn_tile_map_build", "attn_get_status", "attn_shutdown", "tile_map_shape",
            "AttnError", "MASK_NONE", "MASK_CAUSAL", "MASK_WINDOW", "MASK_DOC"]
 
@@ -50,6 +50,22 @@ def attn_fwd(q, k, v, o=None, lse=None, scale=None, mask_kind=MASK_NONE, window=
                       int(mask_kind), int(window), float(softcap), _ptr(alibi_slopes), _ptr(doc_ids),
                       _stream(stream))
     check(rc, "attn_fwd")
+    return o, lse
+
+
+def attn_fwd_noalloc(q, k, v, o, lse, scale=None, mask_kind=MASK_NONE, window=0, softcap=0.0,
+                     alibi_slopes=None, doc_ids=None, stream=None):
+    """attn_fwd without any device allocation inside the call: the caller passes the
+    outputs, and the document-mask tile map uses the library's fixed per-device array
+    (see include/attn.h).  For callers that cannot allocate during the call."""
+    lib = load()
+    B, H, Sq, D = q.shape
+    Sk = k.shape[2]
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    rc = lib.attn_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Sq, Sk, D, float(scale),
+                              int(mask_kind), int(window), float(softcap), _ptr(alibi_slopes), _ptr(doc_ids),
+                              _stream(stream))
+    check(rc, "attn_fwd_noalloc")
     return o, lse
 
 

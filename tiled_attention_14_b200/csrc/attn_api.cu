@@ -234,6 +234,70 @@ int run_fwd(bool fp8, const void* q, const void* k, const void* v, const float* 
   return rc;
 }
 
+// ---------------------------------------------------------------------------------------
+// Allocation-free variant of the document-mask path.
+//
+// Some callers cannot allocate device memory during a call: code that runs inside a
+// framework whose caching allocator owns all of device memory (an outside allocation can
+// fail under its memory cap or fragment its pool), serving loops that must not let an
+// allocation or free synchronise the device in the middle of a request, and programs that
+// reserve a fixed memory budget up front.  For them the tile map that attn_fwd builds in a
+// stream-ordered workspace lives instead in the array below, sized for at most
+// ATTN_NOALLOC_SCRATCH_BYTES.  Every device that loads this library holds the array until
+// the process exits.  The array is shared by all calls on a device: two such calls whose
+// kernels overlap on the GPU (different streams, no ordering between them) race on it.
+// Nothing in it has to start at zero: each call's map build rewrites every value the
+// attention kernel then reads.
+// ---------------------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_noalloc_scratch[ATTN_NOALLOC_SCRATCH_BYTES];
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the array on the current device.  Host code may only use the symbol to
+// look this address up (the symbol itself is a host-side stand-in, not a device pointer);
+// this is done on the first call on each device, with that device current.
+int noalloc_scratch(int dev, void** out) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) return ATTN_ERR_CUDA;
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return ATTN_OK;
+}
+
+int run_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Sq,
+                    int Sk, int D, float scale, int mask_kind, int window, float softcap, const float* alibi,
+                    const int* doc_ids, cudaStream_t stream) {
+  int rc = check_common(q, k, v, o, lse, B, H, Sq, Sk, D, scale, mask_kind, window, softcap, alibi, doc_ids);
+  if (rc != ATTN_OK) return rc;
+  const bool need_map = (mask_kind & ATTN_MASK_DOC) != 0;
+  if (need_map && ws_bytes_for_map(B, Sq, Sk) > static_cast<size_t>(ATTN_NOALLOC_SCRATCH_BYTES))
+    return ATTN_ERR_INVALID;   // the tile map would not fit in the fixed array
+  int dev = 0;
+  if ((rc = current_device(&dev)) != ATTN_OK) return rc;
+  void* scratch = nullptr;
+  if (need_map && (rc = noalloc_scratch(dev, &scratch)) != ATTN_OK) return rc;
+
+  FwdParams p = make_params(o, lse, B, H, Sq, Sk, scale, mask_kind, window, softcap, alibi, doc_ids);
+  CUtensorMap tq, tk, tv;
+  if (encode_map(&tq, q, false, B * H, Sq, D) != ATTN_OK || encode_map(&tk, k, false, B * H, Sk, D) != ATTN_OK ||
+      encode_map(&tv, v, false, B * H, Sk, D) != ATTN_OK)
+    return ATTN_ERR_CUDA;
+  if (need_map) {
+    int* c = static_cast<int*>(scratch);
+    uint32_t* e = reinterpret_cast<uint32_t*>(static_cast<char*>(scratch) + ws_counts_bytes(B, Sq));
+    int* sorted = reinterpret_cast<int*>(static_cast<char*>(scratch) + ws_counts_bytes(B, Sq) + ws_entries_bytes(B, Sq, Sk));
+    if ((rc = launch_tile_map(c, e, B, Sq, Sk, mask_kind, window, doc_ids, stream, sorted)) != ATTN_OK) return rc;
+    p.doc_sorted = sorted;
+    p.map_counts = c;
+    p.map_entries = e;
+  }
+  const bool sc = softcap > 0.f, al = alibi != nullptr;
+  if (D == 128) return launch_fwd_d<128, false>(dev, tq, tk, tv, p, sc, al, stream);
+  return launch_fwd_d<64, false>(dev, tq, tk, tv, p, sc, al, stream);
+}
+
 }  // namespace
 
 extern "C" {
@@ -243,6 +307,13 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
              const int* doc_ids, void* stream) {
   return run_fwd(false, q, k, v, nullptr, nullptr, nullptr, o, lse, B, H, Sq, Sk, D, scale, mask_kind, window,
                  softcap, alibi_slopes, doc_ids, nullptr, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+int attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Sq,
+                     int Sk, int D, float scale, int mask_kind, int window, float softcap,
+                     const float* alibi_slopes, const int* doc_ids, void* stream) {
+  return run_fwd_noalloc(q, k, v, o, lse, B, H, Sq, Sk, D, scale, mask_kind, window, softcap, alibi_slopes,
+                         doc_ids, static_cast<cudaStream_t>(stream));
 }
 
 int attn_fwd_with_map(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Sq,
