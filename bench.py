@@ -32,7 +32,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from attn_workloads import (MASK_CAUSAL, MASK_DOC, MASK_WINDOW, WORKLOADS, alibi_slopes,  # noqa: E402
-                            doc_lengths, make_doc_ids, make_qkv)
+                            doc_lengths, make_doc_ids, make_fp8_source, make_qkv)
 
 METRIC = "attention fwd TFLOP/s and % of B200 dense BF16/FP8 tensor peak, per config"
 L2_BYTES = 126 * 1024 * 1024
@@ -278,8 +278,6 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     w = WORKLOADS[args.workload]
-    if w.fp8:
-        ap.error("the FP8 workloads are timed by bench_fp8 options, not by this leg")
 
     if args.impl == "reference":
         run_reference(args, w)
@@ -298,7 +296,10 @@ def main():
     import tiled_attention_14_b200 as ta
     ta._lib.load()
 
-    q, k, v = make_qkv(w.B, w.H, w.Sq, w.Sk, w.D, seed=rank)
+    if w.fp8:
+        q, k, v = make_fp8_source(w.B, w.H, w.Sq, w.D, seed=rank)
+    else:
+        q, k, v = make_qkv(w.B, w.H, w.Sq, w.Sk, w.D, seed=rank)
     sl = alibi_slopes(w.H) if w.alibi else None
     doc = make_doc_ids(w.B, w.Sq) if w.doc else None
     dev = torch.device("cuda", local)
@@ -310,9 +311,27 @@ def main():
     stream = torch.cuda.current_stream(dev)
     launches_per_step = 2 if w.doc else 1
 
+    quant_ms = None
+    if w.fp8:
+        # e4m3 operands with per-128-row scales, quantised once; the quantiser is timed alone
+        q8, qs = ta.attn_quantize_e4m3(qd, stream=stream)
+        k8, ks = ta.attn_quantize_e4m3(kd, stream=stream)
+        v8, vs = ta.attn_quantize_e4m3(vd, stream=stream)
+        e0q, e1q = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0q.record(stream)
+        for t in (qd, kd, vd):
+            ta.attn_quantize_e4m3(t, stream=stream)
+        e1q.record(stream)
+        torch.cuda.synchronize(dev)
+        quant_ms = e0q.elapsed_time(e1q)
+
     def step():
-        ta.attn_fwd(qd, kd, vd, o=o, lse=lse, scale=w.scale, mask_kind=w.mask_kind, window=w.window,
-                    softcap=w.softcap, alibi_slopes=sld, doc_ids=docd, stream=stream)
+        if w.fp8:
+            ta.attn_fwd_fp8(q8, k8, v8, qs, ks, vs, o=o, lse=lse, scale=w.scale, mask_kind=w.mask_kind,
+                            stream=stream)
+        else:
+            ta.attn_fwd(qd, kd, vd, o=o, lse=lse, scale=w.scale, mask_kind=w.mask_kind, window=w.window,
+                        softcap=w.softcap, alibi_slopes=sld, doc_ids=docd, stream=stream)
 
     for _ in range(args.warmup):
         step()
@@ -359,8 +378,13 @@ def main():
         q2.copy_(qh, non_blocking=True)
         k2.copy_(kh, non_blocking=True)
         v2.copy_(vh, non_blocking=True)
-        ta.attn_fwd(q2, k2, v2, o=o, lse=lse, scale=w.scale, mask_kind=w.mask_kind, window=w.window,
-                    softcap=w.softcap, alibi_slopes=sld, doc_ids=docd, stream=stream)
+        if w.fp8:
+            a8 = [ta.attn_quantize_e4m3(t, stream=stream) for t in (q2, k2, v2)]
+            ta.attn_fwd_fp8(a8[0][0], a8[1][0], a8[2][0], a8[0][1], a8[1][1], a8[2][1], o=o, lse=lse,
+                            scale=w.scale, mask_kind=w.mask_kind, stream=stream)
+        else:
+            ta.attn_fwd(q2, k2, v2, o=o, lse=lse, scale=w.scale, mask_kind=w.mask_kind, window=w.window,
+                        softcap=w.softcap, alibi_slopes=sld, doc_ids=docd, stream=stream)
         oh.copy_(o, non_blocking=True)
         lh.copy_(lse, non_blocking=True)
 
@@ -392,22 +416,29 @@ def main():
         # time per step minus nothing else for analytic masks (one launch per step)
         launch_ms = float(np.mean(per_launch_ms))
         achieved = flops / (launch_ms * 1e-3) / 1e12
+        # FP8 contractions take the FP8 peak: the measured BF16 peak times the nominal
+        # dense FP8 / BF16 ratio (4.5 / 2.25 PFLOP/s)
+        peak = peaks["bf16"] * (2.0 if w.fp8 else 1.0)
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "e4m3" if w.fp8 else "bf16",
             "data": "synthetic", "config": {**workload_config(w), "parallelism": f"replicas x{world}"},
             "tflops_tile_count": tile_count_flops(w) * args.steps * world / (total_ms * 1e-3) / 1e12,
-            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16"], "unit": "TFLOP/s",
-                         "frac": achieved / peaks["bf16"], "traffic": profiled_traffic(args.workload),
-                         "peak_source": f"bf16_tflops of {peaks['source']} peaks (burst); sustained "
-                                        f"{peaks['bf16_sustained']}",
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": profiled_traffic(args.workload),
+                         "peak_source": (f"bf16_tflops of {peaks['source']} peaks (burst)"
+                                         + (" x 2 (nominal fp8/bf16)" if w.fp8 else "")
+                                         + f"; bf16 sustained {peaks['bf16_sustained']}"),
                          "kernel": "attn_fwd_kernel", "algorithmic_flops_per_launch": flops},
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "clocks": clocks.summary(),
             "gpu_launches": launches_per_step * args.steps,
         }
+        if quant_ms is not None:
+            line["quantize_ms_per_tensor_set"] = quant_ms
         if world == 1 and not args.no_cpu_baseline:
             f, dt, desc = oracle_sample(w, args.cpu_budget)
             line["cpu_baseline"] = {"value": f / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),

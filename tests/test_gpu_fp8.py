@@ -1,0 +1,82 @@
+"""GPU parity of the FP8 e4m3 path: attn_quantize_e4m3 (bit-exact against the oracle's
+encoder, tested elsewhere) then attn_fwd_fp8, compared with the fp64 oracle run on the
+DEQUANTISED Q/K/V with an exact softmax (the reading that makes the tolerance about the
+kernel, not about quantising the inputs).
+
+Gate: cosine similarity >= 0.999 over all outputs; LSE within the BF16 path's 1e-3 (the
+scores are exact products of e4m3 values summed in fp32); max|dO| <= 5e-2 wherever the
+softmax-weighted mean of |v|, E_p|v|, is below 1.  In the value channels scaled x20 as
+outliers the rounding of P to e4m3 alone (up to 2^-4 relative per weight) moves O by up to
+0.73 (an oracle-side diagnostic that rounds P the same way shows this floor), so there the
+bound per element is 5e-2 + 2^-4 E_p|v| + 2^-8 |O| (e4m3 P, then bf16 O)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from attn_workloads import MASK_CAUSAL, MASK_NONE, WORKLOADS, make_fp8_source, sample_rows
+from oracle import e4m3
+from oracle.attention import attention_fwd
+from tests.gpu_helpers import TOL_COS_FP8, TOL_LSE_BF16, TOL_O_FP8
+
+pytestmark = pytest.mark.gpu
+
+E4M3_REL = 2.0 ** -4
+BF16_REL = 2.0 ** -8
+
+
+def _fp8_case(B, H, S, D, mask, rows=None, seed=0):
+    import tiled_attention_14_b200 as ta
+    q, k, v = make_fp8_source(B, H, S, D, seed=seed)
+    qd, kd, vd = (t.cuda().contiguous() for t in (q, k, v))
+    q8, qs = ta.attn_quantize_e4m3(qd)
+    k8, ks = ta.attn_quantize_e4m3(kd)
+    v8, vs = ta.attn_quantize_e4m3(vd)
+    scale = 1.0 / math.sqrt(D)
+    o, lse = ta.attn_fwd_fp8(q8, k8, v8, qs, ks, vs, scale=scale, mask_kind=mask)
+    torch.cuda.synchronize()
+    assert ta.attn_get_status() == 0
+    # oracle on the dequantised inputs (its own encoder; bit-identical codes and scales)
+    deq = []
+    for x in (q, k, v):
+        c, s = e4m3.quantize_blocks(x)
+        deq.append(e4m3.dequantize_blocks(c, s))
+    O, L = attention_fwd(deq[0], deq[1], deq[2], scale, mask, rows=rows)
+    Oabs, _ = attention_fwd(deq[0], deq[1], np.abs(deq[2]), scale, mask, rows=rows)   # E_p|v|
+    og = o.float().cpu().numpy().astype(np.float64)
+    lg = lse.cpu().numpy().astype(np.float64)
+    if rows is not None:
+        og, lg = og[:, :, rows], lg[:, :, rows]
+    cos = float((og * O).sum() / (np.linalg.norm(og) * np.linalg.norm(O)))
+    err = np.abs(og - O)
+    excess = float((err - (TOL_O_FP8 + E4M3_REL * Oabs + BF16_REL * np.abs(O))).max())
+    small = Oabs < 1.0
+    d_small = float(err[small].max()) if small.any() else 0.0
+    fin = np.isfinite(L)
+    d_l = float(np.abs(lg[fin] - L[fin]).max())
+    assert cos >= TOL_COS_FP8, cos
+    assert d_small <= TOL_O_FP8, d_small          # the absolute gate wherever E_p|v| < 1
+    assert excess <= 0.0, excess
+    assert d_l <= TOL_LSE_BF16, d_l
+    return cos, float(err.max()), d_l
+
+
+@pytest.mark.parametrize("S,mask", [(256, MASK_NONE), (640, MASK_NONE), (300, MASK_CAUSAL), (777, MASK_CAUSAL)])
+def test_fp8_small_shapes(S, mask):
+    _fp8_case(1, 4, S, 128, mask, seed=S)
+
+
+@pytest.mark.parametrize("name", ["fp8", "fp8_causal"])
+def test_fp8_full_size_sampled_rows(name):
+    w = WORKLOADS[name]
+    rows = sample_rows(w.Sq, 16, seed=2)
+    _fp8_case(w.B, w.H, w.Sq, w.D, w.mask_kind, rows=rows)
+
+
+def test_fp8_rejects_d64():
+    import tiled_attention_14_b200 as ta
+    x = torch.zeros(1, 1, 128, 64, device="cuda", dtype=torch.uint8)
+    s = torch.ones(1, 1, 1, device="cuda")
+    with pytest.raises(ta.AttnError):
+        ta.attn_fwd_fp8(x, x, x, s, s, s)
