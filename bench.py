@@ -94,6 +94,22 @@ def tile_count_flops(w) -> float:
     return 4.0 * w.D * 256 * 128 * tiles * w.B * w.H
 
 
+# ----------------------------------------------------------------------------- ranks
+def max_over_ranks(x: float, dist=None, device="cpu") -> float:
+    """Max of a per-rank time over all ranks (identity without a process group)."""
+    if dist is None:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(flops_per_step: float, steps: int, world: int, ms: float) -> float:
+    """Whole-job TFLOP/s: every rank ran `steps` steps of the same workload; `ms` is the
+    slowest rank's device time."""
+    return flops_per_step * steps * world / (ms * 1e-3) / 1e12
+
+
 # ----------------------------------------------------------------------------- peaks, clocks
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -319,8 +335,8 @@ def main():
         v8, vs = ta.attn_quantize_e4m3(vd, stream=stream)
         e0q, e1q = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0q.record(stream)
-        for t in (qd, kd, vd):
-            ta.attn_quantize_e4m3(t, stream=stream)
+        for t, (t8, ts) in zip((qd, kd, vd), ((q8, qs), (k8, ks), (v8, vs))):
+            ta.attn_quantize_e4m3(t, t8, ts, stream=stream)
         e1q.record(stream)
         torch.cuda.synchronize(dev)
         quant_ms = e0q.elapsed_time(e1q)
@@ -362,11 +378,8 @@ def main():
         raise SystemExit("kernel status error in the timed region")
 
     flops = algorithmic_flops(w)
-    if dist:
-        tt = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
-    value = flops * args.steps * world / (total_ms * 1e-3) / 1e12
+    total_ms = max_over_ranks(total_ms, dist, dev)
+    value = weak_scaling_value(flops, args.steps, world, total_ms)
 
     # ---- end to end through the public API: pinned host inputs in, host outputs back
     qh, kh, vh = (t.pin_memory() for t in (q, k, v))
@@ -401,12 +414,8 @@ def main():
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1)
-    if dist:
-        tt = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
-    e2e_value = flops * e2e_steps * world / (e2e_ms * 1e-3) / 1e12
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
+    e2e_value = weak_scaling_value(flops, e2e_steps, world, e2e_ms)
     h2d = sum(t.numel() * t.element_size() for t in (q, k, v))
     d2h = o.numel() * o.element_size() + lse.numel() * lse.element_size()
 
@@ -425,7 +434,7 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "e4m3" if w.fp8 else "bf16",
             "data": "synthetic", "config": {**workload_config(w), "parallelism": f"replicas x{world}"},
-            "tflops_tile_count": tile_count_flops(w) * args.steps * world / (total_ms * 1e-3) / 1e12,
+            "tflops_tile_count": weak_scaling_value(tile_count_flops(w), args.steps, world, total_ms),
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": profiled_traffic(args.workload),
                          "peak_source": (f"bf16_tflops of {peaks['source']} peaks (burst)"

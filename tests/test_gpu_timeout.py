@@ -1,0 +1,35 @@
+"""Bounded waits: when a signal inside the kernel never comes, the kernel gives up after
+its time limit, records ATTN_ERR_TIMEOUT in the device status word, frees its tensor
+memory and returns — no trap, no hang — and the CUDA context stays usable.
+
+The test hook makes the second softmax group of every CTA skip its first P-ready signal,
+so the MMA issuer's wait for it runs out (limit 200 ms here)."""
+import pytest
+import torch
+
+from attn_workloads import MASK_CAUSAL, make_qkv
+from tests.gpu_helpers import compare, oracle, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def test_skipped_signal_times_out_and_context_survives():
+    import tiled_attention_14_b200 as ta
+    from tiled_attention_14_b200 import _lib
+    lib = _lib.load()
+    q, k, v = make_qkv(1, 2, 640, 640, 128, seed=41)
+    qd, kd, vd = to_dev(q, k, v)
+    assert ta.attn_get_status() == _lib.ATTN_OK
+    lib.attn_debug_set_fault(1, 200)
+    try:
+        ta.attn_fwd(qd, kd, vd, mask_kind=MASK_CAUSAL)
+        assert ta.attn_get_status() == _lib.ATTN_ERR_TIMEOUT
+    finally:
+        lib.attn_debug_set_fault(0, 1000)
+    # the status word was cleared by the read, and the context still runs kernels correctly
+    assert ta.attn_get_status() == _lib.ATTN_OK
+    o, lse = ta.attn_fwd(qd, kd, vd, mask_kind=MASK_CAUSAL)
+    torch.cuda.synchronize()
+    assert ta.attn_get_status() == _lib.ATTN_OK
+    O, L = oracle(q, k, v, 1.0 / 128 ** 0.5, MASK_CAUSAL)
+    compare(o, lse, O, L)

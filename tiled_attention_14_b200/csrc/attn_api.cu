@@ -360,8 +360,12 @@ int attn_quantize_e4m3(const float* x, void* xq, float* scales, int B, int H, in
   const int nsb = (S + 127) / 128;
   const long long grid = static_cast<long long>(B) * H * nsb;
   if (grid > 0x7fffffffLL) return ATTN_ERR_INVALID;
-  attn::quant_e4m3_kernel<<<static_cast<unsigned>(grid), attn::kQuantThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-      x, static_cast<uint8_t*>(xq), scales, S, D, nsb);
+  if (D <= 128)
+    attn::quant_e4m3_kernel<8><<<static_cast<unsigned>(grid), attn::kQuantThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+        x, static_cast<uint8_t*>(xq), scales, S, D, nsb);
+  else
+    attn::quant_e4m3_kernel<16><<<static_cast<unsigned>(grid), attn::kQuantThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+        x, static_cast<uint8_t*>(xq), scales, S, D, nsb);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

@@ -734,7 +734,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const uint32_t t = tcount + i;
         const int kt = tile_kt(it, i);
         const int cls = tile_class(p, it, i, g, kt);
-        if (!wait_bounded(BAR(B_SFULL + g), t & 1, abort_flag, tmo)) { ok = false; break; }
+        // The warp-collective TMEM accesses below need every lane to agree on the outcome.
+        if (!__all_sync(0xffffffffu, wait_bounded(BAR(B_SFULL + g), t & 1, abort_flag, tmo))) { ok = false; break; }
         tc_fence_after();
         if (cls == 0) {
           // Fully masked for this query tile: P = 0, m and l unchanged.
@@ -750,13 +751,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tc_fence_before();
         if (!(p.fault_skip && g == 1 && t == 0)) mbar_arrive(BAR(B_PFULL + g));
       }
-      if (!ok || *abort_flag) {
+      if (!__all_sync(0xffffffffu, ok && !*abort_flag)) {
         ok = false;
         break;
       }
       // ---- epilogue: O / l -> bf16, LSE
       if (it.n > 0) {
-        if (!wait_bounded(BAR(B_ODONE + g), (tcount + it.n - 1) & 1, abort_flag, tmo)) {
+        if (!__all_sync(0xffffffffu, wait_bounded(BAR(B_ODONE + g), (tcount + it.n - 1) & 1, abort_flag, tmo))) {
           ok = false;
           break;
         }
@@ -780,7 +781,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (row < p.Sq) {
           uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
 #pragma unroll
-          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(wv[4 * v], wv[4 * v + 1], wv[4 * v + 2], wv[4 * v + 3]);
+          for (int v = 0; v < 4; ++v) __stcs(dst + v, make_uint4(wv[4 * v], wv[4 * v + 1], wv[4 * v + 2], wv[4 * v + 3]));
         }
       }
       if (row < p.Sq) {
