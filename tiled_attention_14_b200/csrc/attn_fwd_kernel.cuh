@@ -519,6 +519,33 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       uint32_t lidx = 0;     // ring loads issued (K and V alternate)
       uint32_t qcount = 0;   // Q tile pairs issued
       bool ok = true;
+      // L2 prefetch cursor: runs kPrefetchTiles key tiles ahead of the loads along this CTA's
+      // whole schedule, crossing into the next work item (whose query tiles it warms when it
+      // enters it).  Prefetches are issued one tile at a time between the loads: a burst of
+      // them in front of a work item's first loads delays those loads.
+      int pf_r = -1, pf_j = 0;
+      Item pf_it{};
+      pf_it.n = 0;
+      auto prefetch_next = [&]() {
+        while (pf_j >= pf_it.n) {
+          const int w2 = sched_pos(++pf_r, cta, G);
+          if (w2 >= p.num_items) return;
+          pf_it = make_item(p, w2);
+          pf_j = 0;
+          if (pf_it.n > 0) {
+            for (int pn = 0; pn < C::NPANEL; ++pn) {
+              tma_prefetch_l2_3d(&tm_q, pn * C::PANEL_COLS, pf_it.qb * 256, pf_it.bh);
+              tma_prefetch_l2_3d(&tm_q, pn * C::PANEL_COLS, pf_it.qb * 256 + 128, pf_it.bh);
+            }
+          }
+        }
+        const int ktp = tile_kt(pf_it, pf_j++);
+        for (int pn = 0; pn < C::NPANEL; ++pn) {
+          tma_prefetch_l2_3d(&tm_k, pn * C::PANEL_COLS, ktp * 128, pf_it.bh);
+          tma_prefetch_l2_3d(&tm_v, pn * C::PANEL_COLS, ktp * 128, pf_it.bh);
+        }
+      };
+      for (int k = 0; k < kPrefetchTiles; ++k) prefetch_next();
       for (int r = 0; ok; ++r) {
         const int w = sched_pos(r, cta, G);
         if (w >= p.num_items) break;
@@ -537,31 +564,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         if (!ok) break;
         ++qcount;
-        // Warm L2 with the next item's query tiles and first key/value tiles.
-        for (int r2 = r + 1;; ++r2) {
-          const int w2 = sched_pos(r2, cta, G);
-          if (w2 >= p.num_items) break;
-          const Item nx = make_item(p, w2);
-          if (nx.n == 0) continue;
-          for (int pn = 0; pn < C::NPANEL; ++pn) {
-            tma_prefetch_l2_3d(&tm_q, pn * C::PANEL_COLS, nx.qb * 256, nx.bh);
-            tma_prefetch_l2_3d(&tm_q, pn * C::PANEL_COLS, nx.qb * 256 + 128, nx.bh);
-            for (int j = 0; j < min(nx.n, kPrefetchTiles); ++j) {
-              tma_prefetch_l2_3d(&tm_k, pn * C::PANEL_COLS, tile_kt(nx, j) * 128, nx.bh);
-              tma_prefetch_l2_3d(&tm_v, pn * C::PANEL_COLS, tile_kt(nx, j) * 128, nx.bh);
-            }
-          }
-          break;
-        }
         for (int i = 0; i < it.n && ok; ++i) {
           const int kt = tile_kt(it, i);
-          if (i + kPrefetchTiles < it.n) {
-            const int ktp = tile_kt(it, i + kPrefetchTiles);
-            for (int pn = 0; pn < C::NPANEL; ++pn) {
-              tma_prefetch_l2_3d(&tm_k, pn * C::PANEL_COLS, ktp * 128, it.bh);
-              tma_prefetch_l2_3d(&tm_v, pn * C::PANEL_COLS, ktp * 128, it.bh);
-            }
-          }
           for (int kv = 0; kv < 2; ++kv) {
             const uint32_t slot = lidx % C::NS;
             if (!wait_bounded(BAR(B_KVEMPTY + slot), ((lidx / C::NS) & 1) ^ 1, abort_flag, tmo)) {
@@ -575,6 +579,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                           BAR(B_KVFULL + slot), pn * C::PANEL_COLS, kt * 128, it.bh, pol_kv);
             ++lidx;
           }
+          if (ok) prefetch_next();
         }
       }
       // Drain: every copy issued by this thread has landed before the CTA may exit.
