@@ -9,12 +9,15 @@
 //
 // Work item: one (b, h) and one block of 256 query rows, made of two 128-row query tiles
 // (the 256x128 Blackwell tile shape named on the FlexAttention page, section "Aktuelle
-// Einschränkungen").  One CTA per work item, 10 warps:
+// Einschränkungen").  Persistent: one CTA per SM walks a static share of the work items.
+// 12 warps:
 //   warps 0-3  softmax group 0: one thread per row of query tile 0
 //   warps 4-7  softmax group 1: one thread per row of query tile 1
-//   warp  8    TMA producer: Q tiles once, then a ring of K and V tiles
+//   warp  8    TMA producer: the item's Q tiles, then a ring of K and V tiles, and an L2
+//              prefetch cursor a few key tiles ahead
 //   warp  9    MMA issuer (one thread): S_g = Q_g K^T and O_g += P_g V with tcgen05, both
-//              accumulating in tensor memory; also allocates / frees TMEM.
+//              accumulating in tensor memory; also allocates / frees TMEM
+//   warps 10-11 idle (their warpgroup's registers go to the softmax warpgroups).
 // Tensor memory (512 columns): S0 | S1 | O0 | O1.  P_g (bf16 or e4m3) is written over the
 // first columns of S_g once the thread has read its whole S row.
 //
@@ -518,6 +521,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const uint64_t pol_q = policy_evict_first();
       uint32_t lidx = 0;     // ring loads issued (K and V alternate)
       uint32_t qcount = 0;   // Q tile pairs issued
+      uint32_t q_issued[2] = {0, 0};   // loads per query buffer: an abort between the two
+                                       // buffers of a pair still drains the first
       bool ok = true;
       // L2 prefetch cursor: runs kPrefetchTiles key tiles ahead of the loads along this CTA's
       // whole schedule, crossing into the next work item (whose query tiles it warms when it
@@ -561,6 +566,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           for (int pn = 0; pn < C::NPANEL; ++pn)
             tma_load_3d(sbase + C::OFF_Q + g * C::TILE_BYTES + pn * C::PANEL_BYTES, &tm_q,
                         BAR(B_QFULL + g), pn * C::PANEL_COLS, it.qb * 256 + 128 * g, it.bh, pol_q);
+          ++q_issued[g];
         }
         if (!ok) break;
         ++qcount;
@@ -583,10 +589,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
       }
       // Drain: every copy issued by this thread has landed before the CTA may exit.
-      if (qcount > 0) {
-        drain_bounded(BAR(B_QFULL + 0), (qcount - 1) & 1, tmo);
-        drain_bounded(BAR(B_QFULL + 1), (qcount - 1) & 1, tmo);
-      }
+      for (int g = 0; g < 2; ++g)
+        if (q_issued[g] > 0) drain_bounded(BAR(B_QFULL + g), (q_issued[g] - 1) & 1, tmo);
       for (uint32_t idx = (lidx > C::NS ? lidx - C::NS : 0); idx < lidx; ++idx)
         drain_bounded(BAR(B_KVFULL + idx % C::NS), (idx / C::NS) & 1, tmo);
     }
