@@ -323,10 +323,8 @@ __device__ __forceinline__ void softmax_tile(const FwdParams& p, const Item& it,
       auto modify = [&](float t, int c) -> float {
         if constexpr (!kPlain) {
           if constexpr (SOFTCAP) {
-            // tanh(x) = sign(x) (1 - 2 / (e^{2|x|} + 1)): absolute error ~1e-7
-            const float x = t * sc_in;
-            const float e = ex2_approx(fabsf(x) * (2.f * kLog2e));
-            t = copysignf(1.f - 2.f * rcp_approx(e + 1.f), x) * p.sc_out;
+            // one MUFU tanh per score (relative error below 2^-10.98)
+            t = tanh_approx(t * sc_in) * p.sc_out;
           } else {
             t *= sc;
           }
