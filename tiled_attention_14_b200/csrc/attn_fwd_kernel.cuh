@@ -341,12 +341,28 @@ __device__ __forceinline__ void softmax_tile(const FwdParams& p, const Item& it,
         // and, for unsorted document ids, doc[c] == doc of the row
         const int clo = jlo_row - c0, chi = jhi_row - c0;
         if (!has_doc) {
+          // The row's visible columns as a 128-bit mask (four words), built once per tile;
+          // each score then needs one bit test and a select instead of two compares (measured:
+          // document masks +14 %, window +4 %).  With ALiBi the compare form measured 2 %
+          // faster, so that variant keeps it.
+          uint32_t vm[4];
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const int lo = min(max(clo - 32 * w, 0), 32), hi = min(max(chi + 1 - 32 * w, 0), 32);
+            const uint32_t below_hi = hi >= 32 ? 0xffffffffu : ((1u << hi) - 1u);
+            const uint32_t below_lo = lo >= 32 ? 0xffffffffu : ((1u << lo) - 1u);
+            vm[w] = below_hi & ~below_lo;
+          }
+          auto visible = [&](int c) -> bool {
+            if constexpr (ALIBI) return c >= clo && c <= chi;
+            else return ((vm[c >> 5] >> (c & 31)) & 1u) != 0u;
+          };
 #pragma unroll
           for (int c = 0; c < 128; c += 2) {
             float t0 = modify(__uint_as_float(s[c]), c);
             float t1 = modify(__uint_as_float(s[c + 1]), c + 1);
-            t0 = (c >= clo && c <= chi) ? t0 : kNegInf;
-            t1 = (c + 1 >= clo && c + 1 <= chi) ? t1 : kNegInf;
+            t0 = visible(c) ? t0 : kNegInf;
+            t1 = visible(c + 1) ? t1 : kNegInf;
             s[c] = __float_as_uint(t0);
             s[c + 1] = __float_as_uint(t1);
             mxa[(c >> 1) & 7] = fmax3f(mxa[(c >> 1) & 7], t0, t1);
