@@ -306,13 +306,19 @@ __device__ __forceinline__ void softmax_tile(const FwdParams& p, const Item& it,
       tmem_ld_x128_wait(tS, s);
       float sc = p.scale_log2;     // raw score -> log2 units
       float sc_in = p.sc_in;       // raw score -> tanh argument
-      float pv_factor = 1.f;
+      float pv_log2 = 0.f;         // FP8: log2 of the V block's scale relative to v_norm
+      float inv_pvf = 1.f;         // and the inverse of that factor
       if constexpr (FP8) {
         const size_t kb = static_cast<size_t>(it.bh) * p.nsb_k + kt;
         const float sqk = sq_scale * __ldg(p.k_scale + kb);
         sc *= sqk;
         sc_in *= sqk;
-        pv_factor = __ldg(p.v_scale + kb) / v_norm;
+        // P is multiplied by v_scale[kb] / v_norm before its e4m3 rounding; the factor goes
+        // into the exponent (one add per tile instead of a multiply per score) and the row
+        // sum, which is of the unscaled P, takes its inverse once per tile.
+        const float vs = __ldg(p.v_scale + kb);
+        pv_log2 = lg2_approx(vs / v_norm);
+        inv_pvf = v_norm / vs;
       }
       const int c0 = kt * 128;
       // ---- score_mod (log2 units) and mask; row maximum as a shallow max3 tree.  Each
@@ -323,12 +329,13 @@ __device__ __forceinline__ void softmax_tile(const FwdParams& p, const Item& it,
       auto modify = [&](float t, int c) -> float {
         if constexpr (!kPlain) {
           if constexpr (SOFTCAP) {
-            // one MUFU tanh per score (relative error below 2^-10.98)
+            // one MUFU tanh per score (PTX bound 2^-10.98 relative; 9.9e-6 measured on B200)
             t = tanh_approx(t * sc_in) * p.sc_out;
-          } else {
-            t *= sc;
+            if constexpr (ALIBI) t = fmaf(slope_l2, static_cast<float>(c), t + alibi_base);
+          } else if constexpr (ALIBI) {
+            // bias first (an FMA with the column as an immediate), then one FMA for the score
+            t = fmaf(t, sc, fmaf(slope_l2, static_cast<float>(c), alibi_base));
           }
-          if constexpr (ALIBI) t = fmaf(slope_l2, static_cast<float>(c), t + alibi_base);
         }
         return t;
       };
@@ -413,7 +420,7 @@ __device__ __forceinline__ void softmax_tile(const FwdParams& p, const Item& it,
       const float msub = (m_run == kNegInf) ? 0.f : m_run;
       // ---- exponentials, packed two per register (f32x2 FMA / ADD), P to TMEM in two halves
       const float2 sc2 = make_float2(sc, sc);
-      const float2 nm2 = make_float2(-msub, -msub);
+      const float2 nm2 = make_float2(pv_log2 - msub, pv_log2 - msub);
       // 2^a: with kSwExpEvery > 0, one pair in kSwExpEvery goes to the FMA pipes (software
       // exp2); the split depends on the column only, so FULL and PARTIAL tiles agree bit for bit.
       auto pexp = [&](float a, int c) -> float {
@@ -449,14 +456,14 @@ __device__ __forceinline__ void softmax_tile(const FwdParams& p, const Item& it,
           const float2 p01 = make_float2(pexp(a.x, 4 * c4), pexp(a.y, 4 * c4 + 1));
           const float2 p23 = make_float2(pexp(b.x, 4 * c4 + 2), pexp(b.y, 4 * c4 + 3));
           ls[c4 & 3] = fadd2(ls[c4 & 3], fadd2(p01, p23));
-          pk[c4] = pack_e4m3x2(p01.x * pv_factor, p01.y * pv_factor) |
-                   (pack_e4m3x2(p23.x * pv_factor, p23.y * pv_factor) << 16);
+          pk[c4] = pack_e4m3x2(p01.x, p01.y) | (pack_e4m3x2(p23.x, p23.y) << 16);
           if (c4 == 15) tmem_st_x16_nowait<0>(tS, pk);
         }
         tmem_st_x16_wait<16>(tS + 16, pk);
       }
       const float2 l2 = fadd2(fadd2(ls[0], ls[1]), fadd2(ls[2], ls[3]));
-      l_run += l2.x + l2.y;
+      if constexpr (FP8) l_run += (l2.x + l2.y) * inv_pvf;
+      else l_run += l2.x + l2.y;
       // ---- rescale O when the maximum moved by more than TAU (PV_g(i-1) is complete:
       //      its commit preceded the one that signalled S_g(i)).
       if (__any_sync(0xffffffffu, rescale)) {
