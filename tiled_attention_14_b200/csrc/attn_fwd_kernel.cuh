@@ -13,8 +13,8 @@
 // 12 warps:
 //   warps 0-3  softmax group 0: one thread per row of query tile 0
 //   warps 4-7  softmax group 1: one thread per row of query tile 1
-//   warp  8    TMA producer: the item's Q tiles, then a ring of K and V tiles, and an L2
-//              prefetch cursor a few key tiles ahead
+//   warp  8    TMA producer: the item's Q tiles, then a ring of K and V tiles (no L2
+//              prefetches: measured, they delay the loads behind them in the TMA unit)
 //   warp  9    MMA issuer (one thread): S_g = Q_g K^T and O_g += P_g V with tcgen05, both
 //              accumulating in tensor memory; also allocates / frees TMEM
 //   warps 10-11 idle (their warpgroup's registers go to the softmax warpgroups).
@@ -57,7 +57,6 @@ static_assert(256 * kSoftmaxRegs + 128 * kControlRegs == kThreads * kLaunchRegs,
 constexpr int kLoadWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr float kTau = 8.0f;
-constexpr int kPrefetchTiles = 3;      // K/V tiles warmed into L2 ahead of the smem ring
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kNegInf = -__builtin_huge_valf();
@@ -545,33 +544,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       uint32_t q_issued[2] = {0, 0};   // loads per query buffer: an abort between the two
                                        // buffers of a pair still drains the first
       bool ok = true;
-      // L2 prefetch cursor: runs kPrefetchTiles key tiles ahead of the loads along this CTA's
-      // whole schedule, crossing into the next work item (whose query tiles it warms when it
-      // enters it).  Prefetches are issued one tile at a time between the loads: a burst of
-      // them in front of a work item's first loads delays those loads.
-      int pf_r = -1, pf_j = 0;
-      Item pf_it{};
-      pf_it.n = 0;
-      auto prefetch_next = [&]() {
-        while (pf_j >= pf_it.n) {
-          const int w2 = sched_pos(++pf_r, cta, G);
-          if (w2 >= p.num_items) return;
-          pf_it = make_item(p, w2);
-          pf_j = 0;
-          if (pf_it.n > 0) {
-            for (int pn = 0; pn < C::NPANEL; ++pn) {
-              tma_prefetch_l2_3d(&tm_q, pn * C::PANEL_COLS, pf_it.qb * 256, pf_it.bh);
-              tma_prefetch_l2_3d(&tm_q, pn * C::PANEL_COLS, pf_it.qb * 256 + 128, pf_it.bh);
-            }
-          }
-        }
-        const int ktp = tile_kt(pf_it, pf_j++);
-        for (int pn = 0; pn < C::NPANEL; ++pn) {
-          tma_prefetch_l2_3d(&tm_k, pn * C::PANEL_COLS, ktp * 128, pf_it.bh);
-          tma_prefetch_l2_3d(&tm_v, pn * C::PANEL_COLS, ktp * 128, pf_it.bh);
-        }
-      };
-      for (int k = 0; k < kPrefetchTiles; ++k) prefetch_next();
       for (int r = 0; ok; ++r) {
         const int w = sched_pos(r, cta, G);
         if (w >= p.num_items) break;
@@ -606,7 +578,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                           BAR(B_KVFULL + slot), pn * C::PANEL_COLS, kt * 128, it.bh, pol_kv);
             ++lidx;
           }
-          if (ok) prefetch_next();
         }
       }
       // Drain: every copy issued by this thread has landed before the CTA may exit.
