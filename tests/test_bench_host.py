@@ -49,3 +49,33 @@ def test_reference_arm_prints_one_line():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["unit"] == "TFLOP/s" and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_committed_traffic_files_are_well_formed():
+    """Every profiles/traffic_<workload>.json names a known workload, a kernel source hash
+    and positive DRAM byte counts whose sum is the per-launch figure."""
+    pdir = os.path.join(ROOT, "profiles")
+    files = [f for f in os.listdir(pdir) if f.startswith("traffic_") and f.endswith(".json")]
+    assert files
+    for f in files:
+        d = json.load(open(os.path.join(pdir, f)))
+        assert f == f"traffic_{d['workload']}.json" and d["workload"] in bench.WORKLOADS
+        assert len(d["kernel_source_hash"]) == 16
+        assert d["dram_bytes_read"] > 0 and d["dram_bytes_write"] > 0
+        assert d["dram_bytes_per_launch"] == d["dram_bytes_read"] + d["dram_bytes_write"]
+
+
+def test_profiled_traffic_is_gated_by_the_kernel_source_hash(tmp_path, monkeypatch):
+    """A traffic figure is reported only while the kernel sources match the capture."""
+    csrc = tmp_path / "tiled_attention_14_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "k.cuh").write_text("// kernel v1\n")
+    (tmp_path / "profiles").mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h = bench.kernel_source_hash()
+    rec = {"workload": "causal", "kernel_source_hash": h, "dram_bytes_per_launch": 123.0}
+    (tmp_path / "profiles" / "traffic_causal.json").write_text(json.dumps(rec))
+    assert bench.profiled_traffic("causal") == 123.0
+    assert bench.profiled_traffic("long") is None              # no capture for this workload
+    (csrc / "k.cuh").write_text("// kernel v2\n")             # the kernel changed since
+    assert bench.profiled_traffic("causal") is None
