@@ -15,7 +15,7 @@ Definition followed
   (page "FlashAttention 4 ...", section "Γιατί οι πυρήνες προσοχής ..."); the oracle
   returns the log-sum-exp built from those two, LSE_i = m_i + ln(l_i), in natural log.
 
-Readings taken where the pages are silent (each is also listed in the design doc):
+Readings taken where the pages are silent:
 * Layout [B, H, S, D].  Causal alignment is bottom-right: query row i sits at key
   position i' = i + (Sk - Sq).
 * Sliding window W counts the diagonal: causal+window keeps 0 <= i' - j < W; window
