@@ -93,7 +93,7 @@ enum {
  *   alibi_slopes  device fp32 [H], or NULL for no ALiBi
  *   doc_ids  device int32 [B,Sk], required iff the DOC bit is set (then Sq == Sk)
  * With the DOC bit the call builds a tile map in a stream-ordered workspace
- * (cudaMallocAsync / cudaFreeAsync on `stream`) and then runs the attention kernel;
+ * (cudaMallocAsync / cudaFreeAsync on `stream`; B <= 65535) and then runs the attention kernel;
  * fully masked tiles are skipped.  CAUSAL and WINDOW tile ranges are computed in the
  * kernel and need no workspace.  Accumulation is fp32; P is rounded to bf16 for P.V.
  */
@@ -113,7 +113,12 @@ ATTN_API int attn_fwd(const void* q, const void* k, const void* v, void* o, floa
  * needs more (bytes ~ 4*B*ceil(Sq/256)*ceil(Sk/128)) returns ATTN_ERR_INVALID, nothing
  * launched.  Without the DOC bit no scratch is used at all.  The first call on a device
  * looks up the array's device address (cudaGetSymbolAddress, with that device current),
- * so make that first call before any stream capture.  All calls on one device share the
+ * so make that first call before any stream capture.  With CUDA's default lazy module
+ * loading that first call also loads the library's device code onto the device, and
+ * loading allocates device memory for it (the 4 MiB array included): the guarantee of
+ * no allocation holds from the second call on, so make one warm-up call per device
+ * first (or set CUDA_MODULE_LOADING=EAGER, which loads everything at context creation).
+ * A DOC call with B > 65535 returns ATTN_ERR_INVALID.  All calls on one device share the
  * array: calls whose kernels may overlap on the GPU race on it and must be ordered (one
  * stream, or events).  Arguments, outputs and errors as attn_fwd (BF16, D = 64 or 128).
  */

@@ -72,3 +72,25 @@ def test_wrapper_raises_on_missing_library(monkeypatch, tmp_path):
     monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "nope.so"))
     with pytest.raises(RuntimeError):
         _lib.load()
+
+
+def test_tmem_moves_header_is_generated():
+    """csrc/tmem_moves.cuh is what tiled_attention_14_b200/gen_tmem_moves.py writes."""
+    from tiled_attention_14_b200 import gen_tmem_moves
+    assert gen_tmem_moves.main(["--check"]) == 0
+
+
+def test_binding_rejects_host_tensors_and_bad_outputs():
+    """The binding checks tensors before it passes bare pointers to the library."""
+    import torch
+    import tiled_attention_14_b200 as ta
+    q = torch.zeros(1, 1, 128, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        ta.attn_fwd(q, q, q)                         # host tensors: there is no CPU path
+    with pytest.raises(ValueError):
+        ta.attn_fwd_noalloc(q, q, q, None, None)
+    meta = torch.empty(1, 1, 128, 128, dtype=torch.bfloat16, device="meta")
+    with pytest.raises(ValueError):
+        ta.attn_fwd(meta, meta, meta)
+    with pytest.raises(ValueError):
+        ta.attn_quantize_e4m3(torch.zeros(1, 1, 128, 128))

@@ -28,12 +28,55 @@ def _stream(stream):
     return stream.cuda_stream
 
 
+def _need(t, name, dtype, shape, device):
+    """Raises ValueError unless ``t`` is a contiguous tensor of this dtype and shape on
+    ``device``.  The C-ABI receives bare pointers and cannot check sizes itself, so a
+    wrong tensor here would make a kernel read or write out of bounds."""
+    if not isinstance(t, torch.Tensor):
+        raise ValueError(f"{name}: expected a torch tensor, got {type(t).__name__}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.device != device:
+        raise ValueError(f"{name}: on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+
+
+def _check_qkv(q, k, v, dtype):
+    """q [B,H,Sq,D], k and v [B,H,Sk,D] of ``dtype``, contiguous, on one CUDA device."""
+    if not isinstance(q, torch.Tensor) or q.dim() != 4:
+        raise ValueError("q: expected a 4-d tensor [B, H, Sq, D]")
+    if q.device.type != "cuda":
+        raise ValueError(f"q: on {q.device}, expected a CUDA device (there is no CPU path)")
+    B, H, Sq, D = q.shape
+    _need(q, "q", dtype, (B, H, Sq, D), q.device)
+    if not isinstance(k, torch.Tensor) or k.dim() != 4:
+        raise ValueError("k: expected a 4-d tensor [B, H, Sk, D]")
+    Sk = k.shape[2]
+    _need(k, "k", dtype, (B, H, Sk, D), q.device)
+    _need(v, "v", dtype, (B, H, Sk, D), q.device)
+    return B, H, Sq, Sk, D
+
+
+def _check_mods(q, H, B, Sk, alibi_slopes, doc_ids):
+    if alibi_slopes is not None:
+        _need(alibi_slopes, "alibi_slopes", torch.float32, (H,), q.device)
+    if doc_ids is not None:
+        _need(doc_ids, "doc_ids", torch.int32, (B, Sk), q.device)
+
+
 def _out(q, o, lse):
     B, H, Sq, D = q.shape
     if o is None:
         o = torch.empty(B, H, Sq, D, dtype=torch.bfloat16, device=q.device)
+    else:
+        _need(o, "o", torch.bfloat16, (B, H, Sq, D), q.device)
     if lse is None:
         lse = torch.empty(B, H, Sq, dtype=torch.float32, device=q.device)
+    else:
+        _need(lse, "lse", torch.float32, (B, H, Sq), q.device)
     return o, lse
 
 
@@ -42,8 +85,8 @@ def attn_fwd(q, k, v, o=None, lse=None, scale=None, mask_kind=MASK_NONE, window=
     """BF16 attention forward. q [B,H,Sq,D], k/v [B,H,Sk,D] bf16 contiguous on one device.
     Returns (o bf16 [B,H,Sq,D], lse fp32 [B,H,Sq])."""
     lib = load()
-    B, H, Sq, D = q.shape
-    Sk = k.shape[2]
+    B, H, Sq, Sk, D = _check_qkv(q, k, v, torch.bfloat16)
+    _check_mods(q, H, B, Sk, alibi_slopes, doc_ids)
     o, lse = _out(q, o, lse)
     scale = 1.0 / math.sqrt(D) if scale is None else scale
     rc = lib.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Sq, Sk, D, float(scale),
@@ -59,8 +102,11 @@ def attn_fwd_noalloc(q, k, v, o, lse, scale=None, mask_kind=MASK_NONE, window=0,
     outputs, and the document-mask tile map uses the library's fixed per-device array
     (see include/attn.h).  For callers that cannot allocate during the call."""
     lib = load()
-    B, H, Sq, D = q.shape
-    Sk = k.shape[2]
+    B, H, Sq, Sk, D = _check_qkv(q, k, v, torch.bfloat16)
+    _check_mods(q, H, B, Sk, alibi_slopes, doc_ids)
+    if o is None or lse is None:
+        raise ValueError("attn_fwd_noalloc: the caller passes o and lse (nothing is allocated)")
+    _out(q, o, lse)
     scale = 1.0 / math.sqrt(D) if scale is None else scale
     rc = lib.attn_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Sq, Sk, D, float(scale),
                               int(mask_kind), int(window), float(softcap), _ptr(alibi_slopes), _ptr(doc_ids),
@@ -77,6 +123,8 @@ def attn_tile_map_build(B, Sq, Sk, mask_kind, window=0, doc_ids=None, device=Non
     """Returns (counts int32 [B, nqb], entries int32 view of uint32 [B, nqb, nkt])."""
     lib = load()
     device = device if device is not None else (doc_ids.device if doc_ids is not None else "cuda")
+    if doc_ids is not None:
+        _need(doc_ids, "doc_ids", torch.int32, (B, Sk), torch.device(device))
     cs, es = tile_map_shape(B, Sq, Sk)
     counts = torch.empty(cs, dtype=torch.int32, device=device)
     entries = torch.zeros(es, dtype=torch.int32, device=device)
@@ -89,8 +137,11 @@ def attn_tile_map_build(B, Sq, Sk, mask_kind, window=0, doc_ids=None, device=Non
 def attn_fwd_with_map(q, k, v, counts, entries, o=None, lse=None, scale=None, mask_kind=MASK_NONE,
                       window=0, softcap=0.0, alibi_slopes=None, doc_ids=None, stream=None):
     lib = load()
-    B, H, Sq, D = q.shape
-    Sk = k.shape[2]
+    B, H, Sq, Sk, D = _check_qkv(q, k, v, torch.bfloat16)
+    _check_mods(q, H, B, Sk, alibi_slopes, doc_ids)
+    cs, es = tile_map_shape(B, Sq, Sk)
+    _need(counts, "counts", torch.int32, cs, q.device)
+    _need(entries, "entries", torch.int32, es, q.device)
     o, lse = _out(q, o, lse)
     scale = 1.0 / math.sqrt(D) if scale is None else scale
     rc = lib.attn_fwd_with_map(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Sq, Sk, D,
@@ -104,11 +155,18 @@ def attn_fwd_with_map(q, k, v, counts, entries, o=None, lse=None, scale=None, ma
 def attn_quantize_e4m3(x, xq=None, scales=None, stream=None):
     """fp32 [B,H,S,D] -> (e4m3 codes uint8 [B,H,S,D], fp32 scales [B,H,ceil(S/128)])."""
     lib = load()
+    if not isinstance(x, torch.Tensor) or x.dim() != 4 or x.device.type != "cuda":
+        raise ValueError("x: expected a 4-d CUDA tensor [B, H, S, D]")
     B, H, S, D = x.shape
+    _need(x, "x", torch.float32, (B, H, S, D), x.device)
     if xq is None:
         xq = torch.empty(B, H, S, D, dtype=torch.uint8, device=x.device)
+    else:
+        _need(xq, "xq", torch.uint8, (B, H, S, D), x.device)
     if scales is None:
         scales = torch.empty(B, H, (S + 127) // 128, dtype=torch.float32, device=x.device)
+    else:
+        _need(scales, "scales", torch.float32, (B, H, (S + 127) // 128), x.device)
     rc = lib.attn_quantize_e4m3(_ptr(x), _ptr(xq), _ptr(scales), B, H, S, D, _stream(stream))
     check(rc, "attn_quantize_e4m3")
     return xq, scales
@@ -118,8 +176,11 @@ def attn_fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o=None, lse=None, scale=
                  mask_kind=MASK_NONE, window=0, softcap=0.0, alibi_slopes=None, doc_ids=None,
                  stream=None):
     lib = load()
-    B, H, Sq, D = q8.shape
-    Sk = k8.shape[2]
+    B, H, Sq, Sk, D = _check_qkv(q8, k8, v8, torch.uint8)
+    _check_mods(q8, H, B, Sk, alibi_slopes, doc_ids)
+    _need(q_scale, "q_scale", torch.float32, (B, H, (Sq + 127) // 128), q8.device)
+    _need(k_scale, "k_scale", torch.float32, (B, H, (Sk + 127) // 128), q8.device)
+    _need(v_scale, "v_scale", torch.float32, (B, H, (Sk + 127) // 128), q8.device)
     o, lse = _out(q8, o, lse)
     scale = 1.0 / math.sqrt(D) if scale is None else scale
     rc = lib.attn_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(q_scale), _ptr(k_scale), _ptr(v_scale),

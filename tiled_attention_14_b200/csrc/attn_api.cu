@@ -192,6 +192,8 @@ int run_fwd(bool fp8, const void* q, const void* k, const void* v, const float* 
   if (rc != ATTN_OK) return rc;
   if (fp8 && (D != 128 || !qs || !ks || !vs)) return ATTN_ERR_INVALID;
   if ((counts == nullptr) != (entries == nullptr)) return ATTN_ERR_INVALID;
+  // the tile-map build launches one grid row per batch entry (grid.y <= 65535)
+  if (counts == nullptr && (mask_kind & ATTN_MASK_DOC) && B > 65535) return ATTN_ERR_INVALID;
   int dev = 0;
   if ((rc = current_device(&dev)) != ATTN_OK) return rc;
 
@@ -272,6 +274,7 @@ int run_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float*
   int rc = check_common(q, k, v, o, lse, B, H, Sq, Sk, D, scale, mask_kind, window, softcap, alibi, doc_ids);
   if (rc != ATTN_OK) return rc;
   const bool need_map = (mask_kind & ATTN_MASK_DOC) != 0;
+  if (need_map && B > 65535) return ATTN_ERR_INVALID;   // tile-map grid.y = B
   if (need_map && ws_bytes_for_map(B, Sq, Sk) > static_cast<size_t>(ATTN_NOALLOC_SCRATCH_BYTES))
     return ATTN_ERR_INVALID;   // the tile map would not fit in the fixed array
   int dev = 0;
