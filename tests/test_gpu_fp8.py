@@ -5,10 +5,12 @@ kernel, not about quantising the inputs).
 
 Gate: cosine similarity >= 0.999 over all outputs; LSE within the BF16 path's 1e-3 (the
 scores are exact products of e4m3 values summed in fp32); max|dO| <= 5e-2 wherever the
-softmax-weighted mean of |v|, E_p|v|, is below 1.  In the value channels scaled x20 as
-outliers the rounding of P to e4m3 alone (up to 2^-4 relative per weight) moves O by up to
-0.73 (an oracle-side diagnostic that rounds P the same way shows this floor), so there the
-bound per element is 5e-2 + 2^-4 E_p|v| + 2^-8 |O| (e4m3 P, then bf16 O)."""
+softmax-weighted mean of |v|, E_p|v|, is below 1.  Rounding P to e4m3 is a step of the
+method and alone moves O by more than 5e-2 in the x20 value channels of rows with few
+keys (tests/test_oracle_fp8_floor.py shows it on the benchmark inputs), so every element
+is held to 5e-2 + min(W, 6 sigma) + 2^-8 |O|, with W and sigma the worst-case bound and the
+standard deviation of that rounding error for the element (tests/fp8_floor.py) and 2^-8 |O|
+for the bf16 output."""
 import math
 
 import numpy as np
@@ -18,11 +20,11 @@ import torch
 from attn_workloads import MASK_CAUSAL, MASK_NONE, WORKLOADS, make_fp8_source, sample_rows
 from oracle import e4m3
 from oracle.attention import attention_fwd
+from tests.fp8_floor import head_inputs, rounding_bounds
 from tests.gpu_helpers import TOL_COS_FP8, TOL_LSE_BF16, TOL_O_FP8
 
 pytestmark = pytest.mark.gpu
 
-E4M3_REL = 2.0 ** -4
 BF16_REL = 2.0 ** -8
 
 
@@ -38,26 +40,33 @@ def _fp8_case(B, H, S, D, mask, rows=None, seed=0):
     torch.cuda.synchronize()
     assert ta.attn_get_status() == 0
     # oracle on the dequantised inputs (its own encoder; bit-identical codes and scales)
-    deq = []
-    for x in (q, k, v):
-        c, s = e4m3.quantize_blocks(x)
-        deq.append(e4m3.dequantize_blocks(c, s))
+    quant = [e4m3.quantize_blocks(x) for x in (q, k, v)]
+    deq = [e4m3.dequantize_blocks(c, s) for c, s in quant]
     O, L = attention_fwd(deq[0], deq[1], deq[2], scale, mask, rows=rows)
-    Oabs, _ = attention_fwd(deq[0], deq[1], np.abs(deq[2]), scale, mask, rows=rows)   # E_p|v|
+    R = S if rows is None else len(rows)
+    rr = np.arange(S) if rows is None else rows
+    W = np.zeros((B, H, R, D))
+    sig = np.zeros((B, H, R, D))
+    eav = np.zeros((B, H, R, D))
+    for b in range(B):
+        for h in range(H):
+            args = [a for c, s in quant for a in (c[b, h], s[b, h])]
+            qd, kd, vcode, sv = head_inputs(*args)
+            W[b, h], sig[b, h], eav[b, h] = rounding_bounds(qd, kd, vcode, sv, scale, rr, mask)
     og = o.float().cpu().numpy().astype(np.float64)
     lg = lse.cpu().numpy().astype(np.float64)
     if rows is not None:
         og, lg = og[:, :, rows], lg[:, :, rows]
     cos = float((og * O).sum() / (np.linalg.norm(og) * np.linalg.norm(O)))
     err = np.abs(og - O)
-    excess = float((err - (TOL_O_FP8 + E4M3_REL * Oabs + BF16_REL * np.abs(O))).max())
-    small = Oabs < 1.0
+    excess = float((err - (TOL_O_FP8 + np.minimum(W, 6.0 * sig) + BF16_REL * np.abs(O))).max())
+    small = eav < 1.0
     d_small = float(err[small].max()) if small.any() else 0.0
     fin = np.isfinite(L)
     d_l = float(np.abs(lg[fin] - L[fin]).max())
     assert cos >= TOL_COS_FP8, cos
     assert d_small <= TOL_O_FP8, d_small          # the absolute gate wherever E_p|v| < 1
-    assert excess <= 0.0, excess
+    assert excess <= 0.0, excess                  # the rounding-of-P bound everywhere
     assert d_l <= TOL_LSE_BF16, d_l
     return cos, float(err.max()), d_l
 
