@@ -112,12 +112,25 @@ def weak_scaling_value(flops_per_step: float, steps: int, world: int, ms: float)
 
 # ----------------------------------------------------------------------------- peaks, clocks
 def measured_peaks():
+    """Roofline denominators.  BF16 and HBM from MEASURED_PEAKS.json (written on this pool's
+    B200s); FP8 e4m3 from profiles/fp8_peak.json (written by ``bench.py --measure-fp8-peak``
+    on a B200), else the BF16 figure times the nominal dense FP8/BF16 ratio (4.5 / 2.25)."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         d = json.load(open(p))
-        return {"bf16": d["bf16_tflops"], "bf16_sustained": d.get("bf16_tflops_sustained"),
-                "hbm": d["hbm_gbs"], "source": "measured"}
-    return {"bf16": 1590.0, "bf16_sustained": 1400.0, "hbm": 6650.0, "source": "fallback"}
+        out = {"bf16": d["bf16_tflops"], "bf16_sustained": d.get("bf16_tflops_sustained"),
+               "hbm": d["hbm_gbs"], "source": "measured"}
+    else:
+        out = {"bf16": 1590.0, "bf16_sustained": 1400.0, "hbm": 6650.0, "source": "fallback"}
+    f = os.path.join(ROOT, "profiles", "fp8_peak.json")
+    if os.path.exists(f):
+        d = json.load(open(f))
+        out.update(fp8=d["fp8_tflops"], fp8_sustained=d.get("fp8_tflops_sustained"),
+                   fp8_source="measured e4m3 GEMM (profiles/fp8_peak.json)")
+    else:
+        out.update(fp8=out["bf16"] * 2.0, fp8_sustained=(out["bf16_sustained"] or 0.0) * 2.0,
+                   fp8_source="bf16 x 2 (nominal dense fp8/bf16 ratio)")
+    return out
 
 
 class ClockSampler:
@@ -281,6 +294,176 @@ def workload_config(w):
 
 
 # ----------------------------------------------------------------------------- GPU leg
+class Case:
+    """One workload resident on the device: its inputs, outputs and a step() that runs the
+    whole hot path once through the public API (tile map + attention for documents)."""
+
+    def __init__(self, ta, w, dev, seed):
+        self.w, self.ta, self.dev = w, ta, dev
+        self.stream = torch.cuda.current_stream(dev)
+        if w.fp8:
+            self.host = make_fp8_source(w.B, w.H, w.Sq, w.D, seed=seed)
+        else:
+            self.host = make_qkv(w.B, w.H, w.Sq, w.Sk, w.D, seed=seed)
+        self.q, self.k, self.v = (t.to(dev).contiguous() for t in self.host)
+        sl = alibi_slopes(w.H) if w.alibi else None
+        doc = make_doc_ids(w.B, w.Sq) if w.doc else None
+        self.sl = None if sl is None else sl.to(dev)
+        self.doc = None if doc is None else doc.to(dev)
+        self.o = torch.empty(w.B, w.H, w.Sq, w.D, dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty(w.B, w.H, w.Sq, dtype=torch.float32, device=dev)
+        self.launches_per_step = 2 if w.doc else 1
+        if w.fp8:
+            # e4m3 operands with per-128-row scales, quantised once (the quantiser is timed alone)
+            self.q8 = [ta.attn_quantize_e4m3(t, stream=self.stream) for t in (self.q, self.k, self.v)]
+
+    def step(self):
+        w, ta = self.w, self.ta
+        if w.fp8:
+            (q8, qs), (k8, ks), (v8, vs) = self.q8
+            ta.attn_fwd_fp8(q8, k8, v8, qs, ks, vs, o=self.o, lse=self.lse, scale=w.scale,
+                            mask_kind=w.mask_kind, stream=self.stream)
+        else:
+            ta.attn_fwd(self.q, self.k, self.v, o=self.o, lse=self.lse, scale=w.scale, mask_kind=w.mask_kind,
+                        window=w.window, softcap=w.softcap, alibi_slopes=self.sl, doc_ids=self.doc,
+                        stream=self.stream)
+
+    def quantize_ms(self, reps=5):
+        ta = self.ta
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(self.stream)
+        for _ in range(reps):
+            for t, (t8, ts) in zip((self.q, self.k, self.v), self.q8):
+                ta.attn_quantize_e4m3(t, t8, ts, stream=self.stream)
+        e1.record(self.stream)
+        torch.cuda.synchronize(self.dev)
+        return e0.elapsed_time(e1) / reps
+
+    def tile_map_ms(self, reps=20):
+        w, ta = self.w, self.ta
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(self.stream)
+        for _ in range(reps):
+            ta.attn_tile_map_build(w.B, w.Sq, w.Sk, w.mask_kind, w.window, doc_ids=self.doc, device=self.dev,
+                                   stream=self.stream)
+        e1.record(self.stream)
+        torch.cuda.synchronize(self.dev)
+        return e0.elapsed_time(e1) / reps
+
+
+def time_launches(step, n, stream, dev, flush=None):
+    """Per-launch device times (ms) of n steps, each bracketed by events on the launching
+    stream; with ``flush`` (a buffer larger than L2) L2 is overwritten before every step."""
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    for i in range(n):
+        if flush is not None:
+            flush.add_(1)
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize(dev)
+    return [s.elapsed_time(e) for s, e in zip(starts, ends)]
+
+
+def compulsory_bytes(w) -> int:
+    """Bytes each launch must move at least: Q, K, V read once, O and LSE written once."""
+    eb = 1 if w.fp8 else 2
+    qkv = w.B * w.H * (w.Sq + 2 * w.Sk) * w.D * eb
+    scales = 3 * w.B * w.H * ((w.Sk + 127) // 128) * 4 if w.fp8 else 0
+    return qkv + scales + w.B * w.H * w.Sq * (w.D * 2 + 4)
+
+
+def per_config_record(ta, name, dev, peaks, min_ms=60.0, min_launches=10):
+    """Device time, exact TFLOP/s, roofline fraction and (where profiled) DRAM traffic of one
+    workload, measured alone after 3 warm-up launches."""
+    w = WORKLOADS[name]
+    case = Case(ta, w, dev, seed=0)
+    for _ in range(3):
+        case.step()
+    torch.cuda.synchronize(dev)
+    t1 = time_launches(case.step, 2, case.stream, dev)
+    n = max(min_launches, int(min_ms / max(min(t1), 1e-3)))
+    flush = None
+    if compulsory_bytes(w) < L2_BYTES:
+        flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    ms = time_launches(case.step, n, case.stream, dev, flush)
+    if ta.attn_get_status(case.stream) != 0:
+        raise SystemExit(f"kernel status error in workload {name}")
+    mean_ms = float(np.mean(ms))
+    flops = algorithmic_flops(w)
+    tflops = flops / (mean_ms * 1e-3) / 1e12
+    peak = peaks["fp8"] if w.fp8 else peaks["bf16"]
+    gbs = compulsory_bytes(w) / (mean_ms * 1e-3) / 1e9
+    rec = {"workload": w.note, "launches": n, "ms": mean_ms, "ms_min": float(np.min(ms)),
+           "tflops_exact": tflops, "peak_tflops": peak, "frac": tflops / peak,
+           "dtype": "e4m3" if w.fp8 else "bf16", "compulsory_bytes": compulsory_bytes(w),
+           "gbs_compulsory": gbs, "hbm_frac": gbs / peaks["hbm"],
+           "l2": "flushed before every launch" if flush is not None else "inputs larger than L2",
+           "traffic": profiled_traffic(name)}
+    if w.doc:
+        rec["tile_map_ms"] = case.tile_map_ms()
+        rec["attention_ms"] = mean_ms - rec["tile_map_ms"]
+    if w.fp8:
+        rec["quantize_ms_per_tensor_set"] = case.quantize_ms()
+    del case, flush
+    torch.cuda.empty_cache()
+    return rec
+
+
+def sustained_record(case, dev, peaks, local, seconds=1.5):
+    """Back-to-back launches for about ``seconds`` (long enough for the power cap to act),
+    with its own NVML clock record, against the sustained peak."""
+    t = time_launches(case.step, 3, case.stream, dev)
+    n = max(20, int(seconds * 1e3 / max(float(np.mean(t)), 1e-3)))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local, period_s=0.02) as clocks:
+        e0.record(case.stream)
+        for _ in range(n):
+            case.step()
+        e1.record(case.stream)
+        torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1)
+    tflops = algorithmic_flops(case.w) * n / (ms * 1e-3) / 1e12
+    peak = peaks["fp8_sustained"] if case.w.fp8 else peaks["bf16_sustained"]
+    return {"launches": n, "ms_total": ms, "tflops_exact": tflops, "peak_tflops": peak,
+            "frac": tflops / peak if peak else None,
+            "peak_source": "sustained GEMM peak (back-to-back loop under the power cap)",
+            "clocks": clocks.summary()}
+
+
+def measure_fp8_peak():
+    """Dense e4m3 GEMM throughput on this GPU (torch._scaled_mm, 8192^3, bf16 output):
+    burst = best of 10 single launches after warm-up, sustained = a 4 s back-to-back loop.
+    Prints one JSON line; its numbers go to profiles/fp8_peak.json."""
+    dev = torch.device("cuda", 0)
+    n = 8192
+    g = torch.Generator(device=dev).manual_seed(0)
+    a = torch.randn(n, n, device=dev, generator=g).to(torch.float8_e4m3fn)
+    b = torch.randn(n, n, device=dev, generator=g).to(torch.float8_e4m3fn).t()
+    one = torch.ones((), device=dev)
+    mm = lambda: torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+    for _ in range(10):
+        mm()
+    torch.cuda.synchronize()
+    best = min(time_launches(mm, 10, torch.cuda.current_stream(), dev))
+    flops = 2.0 * n ** 3
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = max(10, int(4000.0 / best))
+    with ClockSampler(0, period_s=0.05) as clocks:
+        e0.record()
+        for _ in range(reps):
+            mm()
+        e1.record()
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    print(json.dumps({"fp8_tflops": flops / (best * 1e-3) / 1e12,
+                      "fp8_tflops_sustained": flops * reps / (ms * 1e-3) / 1e12,
+                      "method": "torch._scaled_mm e4m3 x e4m3 -> bf16, 8192^3; burst best of 10, "
+                                f"sustained {reps} back to back ({ms / 1e3:.1f} s)",
+                      "clocks": clocks.summary(), "gpu": torch.cuda.get_device_name(0)}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -290,13 +473,25 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true", help="skip the per-workload records")
+    ap.add_argument("--measure-fp8-peak", action="store_true", help="time a dense e4m3 GEMM and exit")
+    ap.add_argument("--kernel-only", action="store_true",
+                    help="time the device steps only (no e2e, sustained, per-config or CPU legs): "
+                         "the command the ncu captures run")
+    ap.add_argument("--heads", type=int, default=0, help="override H (smaller ncu captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     w = WORKLOADS[args.workload]
+    if args.heads > 0:
+        import dataclasses
+        w = dataclasses.replace(w, H=args.heads, note=w.note.replace(f"H{w.H}", f"H{args.heads}"))
 
     if args.impl == "reference":
         run_reference(args, w)
+        return
+    if args.measure_fp8_peak:
+        measure_fp8_peak()
         return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -311,46 +506,13 @@ def main():
 
     import tiled_attention_14_b200 as ta
     ta._lib.load()
-
-    if w.fp8:
-        q, k, v = make_fp8_source(w.B, w.H, w.Sq, w.D, seed=rank)
-    else:
-        q, k, v = make_qkv(w.B, w.H, w.Sq, w.Sk, w.D, seed=rank)
-    sl = alibi_slopes(w.H) if w.alibi else None
-    doc = make_doc_ids(w.B, w.Sq) if w.doc else None
     dev = torch.device("cuda", local)
-    qd, kd, vd = (t.to(dev).contiguous() for t in (q, k, v))
-    sld = None if sl is None else sl.to(dev)
-    docd = None if doc is None else doc.to(dev)
-    o = torch.empty(w.B, w.H, w.Sq, w.D, dtype=torch.bfloat16, device=dev)
-    lse = torch.empty(w.B, w.H, w.Sq, dtype=torch.float32, device=dev)
-    stream = torch.cuda.current_stream(dev)
-    launches_per_step = 2 if w.doc else 1
-
-    quant_ms = None
-    if w.fp8:
-        # e4m3 operands with per-128-row scales, quantised once; the quantiser is timed alone
-        q8, qs = ta.attn_quantize_e4m3(qd, stream=stream)
-        k8, ks = ta.attn_quantize_e4m3(kd, stream=stream)
-        v8, vs = ta.attn_quantize_e4m3(vd, stream=stream)
-        e0q, e1q = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0q.record(stream)
-        for t, (t8, ts) in zip((qd, kd, vd), ((q8, qs), (k8, ks), (v8, vs))):
-            ta.attn_quantize_e4m3(t, t8, ts, stream=stream)
-        e1q.record(stream)
-        torch.cuda.synchronize(dev)
-        quant_ms = e0q.elapsed_time(e1q)
-
-    def step():
-        if w.fp8:
-            ta.attn_fwd_fp8(q8, k8, v8, qs, ks, vs, o=o, lse=lse, scale=w.scale, mask_kind=w.mask_kind,
-                            stream=stream)
-        else:
-            ta.attn_fwd(qd, kd, vd, o=o, lse=lse, scale=w.scale, mask_kind=w.mask_kind, window=w.window,
-                        softcap=w.softcap, alibi_slopes=sld, doc_ids=docd, stream=stream)
+    case = Case(ta, w, dev, seed=rank)
+    stream = case.stream
+    quant_ms = case.quantize_ms() if w.fp8 else None
 
     for _ in range(args.warmup):
-        step()
+        case.step()
     torch.cuda.synchronize(dev)
     if ta.attn_get_status(stream) != 0:
         raise SystemExit("kernel status error during warm-up")
@@ -366,7 +528,7 @@ def main():
         t_begin.record(stream)
         for i in range(args.steps):
             starts[i].record(stream)
-            step()
+            case.step()
             ends[i].record(stream)
         t_end.record(stream)
         torch.cuda.synchronize(dev)
@@ -380,12 +542,22 @@ def main():
     flops = algorithmic_flops(w)
     total_ms = max_over_ranks(total_ms, dist, dev)
     value = weak_scaling_value(flops, args.steps, world, total_ms)
+    if args.kernel_only:
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+                              "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+                              "config": workload_config(w), "kernel_only": True,
+                              "gpu_launches": case.launches_per_step * args.steps}), flush=True)
+        if dist:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
 
     # ---- end to end through the public API: pinned host inputs in, host outputs back
-    qh, kh, vh = (t.pin_memory() for t in (q, k, v))
-    oh = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-    lh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-    q2, k2, v2 = (torch.empty_like(t) for t in (qd, kd, vd))
+    qh, kh, vh = (t.pin_memory() for t in case.host)
+    oh = torch.empty(case.o.shape, dtype=case.o.dtype).pin_memory()
+    lh = torch.empty(case.lse.shape, dtype=case.lse.dtype).pin_memory()
+    q2, k2, v2 = (torch.empty_like(t) for t in (case.q, case.k, case.v))
 
     def e2e_step():
         q2.copy_(qh, non_blocking=True)
@@ -393,13 +565,13 @@ def main():
         v2.copy_(vh, non_blocking=True)
         if w.fp8:
             a8 = [ta.attn_quantize_e4m3(t, stream=stream) for t in (q2, k2, v2)]
-            ta.attn_fwd_fp8(a8[0][0], a8[1][0], a8[2][0], a8[0][1], a8[1][1], a8[2][1], o=o, lse=lse,
+            ta.attn_fwd_fp8(a8[0][0], a8[1][0], a8[2][0], a8[0][1], a8[1][1], a8[2][1], o=case.o, lse=case.lse,
                             scale=w.scale, mask_kind=w.mask_kind, stream=stream)
         else:
-            ta.attn_fwd(q2, k2, v2, o=o, lse=lse, scale=w.scale, mask_kind=w.mask_kind, window=w.window,
-                        softcap=w.softcap, alibi_slopes=sld, doc_ids=docd, stream=stream)
-        oh.copy_(o, non_blocking=True)
-        lh.copy_(lse, non_blocking=True)
+            ta.attn_fwd(q2, k2, v2, o=case.o, lse=case.lse, scale=w.scale, mask_kind=w.mask_kind,
+                        window=w.window, softcap=w.softcap, alibi_slopes=case.sl, doc_ids=case.doc, stream=stream)
+        oh.copy_(case.o, non_blocking=True)
+        lh.copy_(case.lse, non_blocking=True)
 
     e2e_steps = max(3, min(args.steps, 20))
     for _ in range(3):
@@ -416,18 +588,16 @@ def main():
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
     e2e_value = weak_scaling_value(flops, e2e_steps, world, e2e_ms)
-    h2d = sum(t.numel() * t.element_size() for t in (q, k, v))
-    d2h = o.numel() * o.element_size() + lse.numel() * lse.element_size()
+    h2d = sum(t.numel() * t.element_size() for t in case.host)
+    d2h = case.o.numel() * case.o.element_size() + case.lse.numel() * case.lse.element_size()
+    del q2, k2, v2, qh, kh, vh, oh, lh
 
     if rank == 0:
         peaks = measured_peaks()
-        # the attention kernel is the dominant launch; its time per launch is the event
-        # time per step minus nothing else for analytic masks (one launch per step)
+        # the attention kernel is the dominant launch (one launch per step for analytic masks)
         launch_ms = float(np.mean(per_launch_ms))
         achieved = flops / (launch_ms * 1e-3) / 1e12
-        # FP8 contractions take the FP8 peak: the measured BF16 peak times the nominal
-        # dense FP8 / BF16 ratio (4.5 / 2.25 PFLOP/s)
-        peak = peaks["bf16"] * (2.0 if w.fp8 else 1.0)
+        peak = peaks["fp8"] if w.fp8 else peaks["bf16"]
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
@@ -437,17 +607,23 @@ def main():
             "tflops_tile_count": weak_scaling_value(tile_count_flops(w), args.steps, world, total_ms),
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": profiled_traffic(args.workload),
-                         "peak_source": (f"bf16_tflops of {peaks['source']} peaks (burst)"
-                                         + (" x 2 (nominal fp8/bf16)" if w.fp8 else "")
-                                         + f"; bf16 sustained {peaks['bf16_sustained']}"),
+                         "peak_source": (peaks["fp8_source"] if w.fp8 else
+                                         f"bf16_tflops of {peaks['source']} peaks (burst)")
+                                        + f"; bf16 sustained {peaks['bf16_sustained']}",
                          "kernel": "attn_fwd_kernel", "algorithmic_flops_per_launch": flops},
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "clocks": clocks.summary(),
-            "gpu_launches": launches_per_step * args.steps,
+            "gpu_launches": case.launches_per_step * args.steps,
         }
         if quant_ms is not None:
             line["quantize_ms_per_tensor_set"] = quant_ms
+        if world == 1:
+            line["sustained"] = sustained_record(case, dev, peaks, local)
+        if world == 1 and not args.no_per_config:
+            del case
+            torch.cuda.empty_cache()
+            line["per_config"] = {name: per_config_record(ta, name, dev, peaks) for name in WORKLOADS}
         if world == 1 and not args.no_cpu_baseline:
             f, dt, desc = oracle_sample(w, args.cpu_budget)
             line["cpu_baseline"] = {"value": f / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),

@@ -11,7 +11,9 @@ it and has no CPU fallback.
 
 Modules
 -------
-``attention``  the attention forward (scores, score_mod, mask, softmax, O, LSE).
+``attention``  the attention forward (scores, score_mod, mask, softmax, O, LSE), with
+               grouped-query heads and packed variable-length sequences.
+``attention_bwd``  the gradients dQ, dK, dV of that forward (the chain rule, step by step).
 ``e4m3``       the FP8 e4m3 code book, encoder and per-128-row block quantiser.
 ``tile_map``   the block-sparse tile classification (EMPTY / PARTIAL / FULL), by brute force.
 

@@ -94,7 +94,9 @@ def attention_fwd(q, k, v, scale: float, mask_kind: int = 0, window: int = 0,
                   chunk: int = 512):
     """fp64 attention forward.
 
-    q: [B,H,Sq,D], k, v: [B,H,Sk,D] (any float dtype; converted exactly to float64).
+    q: [B,H,Sq,D], k, v: [B,Hkv,Sk,D] (any float dtype; converted exactly to float64).
+    Hkv divides H: query head h reads key/value head h // (H // Hkv) (grouped-query
+    attention; Hkv = 1 is multi-query attention, Hkv = H plain multi-head attention).
     alibi_slopes: None or [H].  doc_ids: None or int [B, S] (Sq == Sk).
     rows: None for every query row, else a 1-D array of query rows to evaluate (rows are
     independent given the full K and V, so a subset is exact for those rows).
@@ -104,7 +106,10 @@ def attention_fwd(q, k, v, scale: float, mask_kind: int = 0, window: int = 0,
     k = _f64(k)
     v = _f64(v)
     B, H, Sq, D = q.shape
-    Sk = k.shape[2]
+    Hkv, Sk = k.shape[1], k.shape[2]
+    if H % Hkv != 0:
+        raise ValueError("the number of key/value heads must divide the number of query heads")
+    group = H // Hkv
     if mask_kind & MASK_DOC and Sq != Sk:
         raise ValueError("document mask needs Sq == Sk")
     rows = np.arange(Sq, dtype=np.int64) if rows is None else np.asarray(rows, dtype=np.int64)
@@ -121,11 +126,43 @@ def attention_fwd(q, k, v, scale: float, mask_kind: int = 0, window: int = 0,
             vis = visible_mask(rr, Sq, Sk, mask_kind, window, doc_row)
             for h in range(H):
                 slope = None if slopes is None else slopes[h]
-                s = modified_scores(q[b, h, rr], k[b, h], scale, rr, Sq, Sk, softcap, slope)
+                hk = h // group
+                s = modified_scores(q[b, h, rr], k[b, hk], scale, rr, Sq, Sk, softcap, slope)
                 P, m, l = softmax_rows(s, vis)
-                O[b, h, r0:r0 + len(rr)] = P @ v[b, h]
+                O[b, h, r0:r0 + len(rr)] = P @ v[b, hk]
                 with np.errstate(divide="ignore"):
                     LSE[b, h, r0:r0 + len(rr)] = np.where(l > 0, m + np.log(l), -np.inf)
+    return O, LSE
+
+
+def attention_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, scale: float, mask_kind: int = 0,
+                         window: int = 0, softcap: float = 0.0, alibi_slopes=None):
+    """fp64 attention over packed variable-length sequences.
+
+    Sequence s holds query tokens cu_seqlens_q[s] .. cu_seqlens_q[s+1]-1 and key tokens
+    cu_seqlens_k[s] .. cu_seqlens_k[s+1]-1; it attends only within itself, exactly as a
+    separate batch entry of its own lengths would (masks, causal alignment and ALiBi
+    positions are per sequence).  Token-major layout: q [Tq, H, D], k, v [Tk, Hkv, D].
+    Returns (O [Tq, H, D], LSE [H, Tq]) in float64; tokens of no sequence stay O = 0,
+    LSE = -inf."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    cq = np.asarray(cu_seqlens_q, dtype=np.int64).reshape(-1)
+    ck = np.asarray(cu_seqlens_k, dtype=np.int64).reshape(-1)
+    Tq, H, D = q.shape
+    O = np.zeros((Tq, H, D), dtype=np.float64)
+    LSE = np.full((H, Tq), -np.inf, dtype=np.float64)
+    for s in range(len(cq) - 1):
+        q0, q1, k0, k1 = cq[s], cq[s + 1], ck[s], ck[s + 1]
+        if q1 <= q0:
+            continue
+        if k1 <= k0:
+            continue
+        qs = q[q0:q1].transpose(1, 0, 2)[None]
+        ks = k[k0:k1].transpose(1, 0, 2)[None]
+        vs = v[k0:k1].transpose(1, 0, 2)[None]
+        o, lse = attention_fwd(qs, ks, vs, scale, mask_kind, window, softcap, alibi_slopes)
+        O[q0:q1] = o[0].transpose(1, 0, 2)
+        LSE[:, q0:q1] = lse[0]
     return O, LSE
 
 
