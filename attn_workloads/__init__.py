@@ -42,6 +42,12 @@ class Workload:
     doc: bool = False
     fp8: bool = False
     note: str = ""
+    Hkv: int = 0             # key/value heads (0: same as H)
+    varlen: bool = False     # packed sequences with the document lengths of doc_lengths()
+
+    @property
+    def kv_heads(self) -> int:
+        return self.Hkv or self.H
 
     @property
     def scale(self) -> float:
@@ -67,17 +73,32 @@ WORKLOADS = {
                     note="B2 H16 S16384 D128 FP8 e4m3, non-causal"),
     "fp8_causal": Workload("fp8_causal", 2, 16, 16384, 16384, 128, MASK_CAUSAL, fp8=True,
                            note="B2 H16 S16384 D128 FP8 e4m3, causal"),
+    # Beyond the five configurations: grouped-query heads and packed sequences (the two
+    # gaps the FA4 page names), on shapes of the configurations above.
+    "gqa": Workload("gqa", 4, 32, 4096, 4096, 128, MASK_CAUSAL, Hkv=8,
+                    note="B4 H32 Hkv8 S4096 D128 causal (grouped-query heads)"),
+    "varlen": Workload("varlen", 2, 16, 8192, 8192, 128, MASK_NONE, varlen=True,
+                       note="2 x 8192 tokens packed as sequences of lengths U[256,2048], H16 D128"),
 }
 
 
+def varlen_cu_seqlens(B: int, S: int) -> torch.Tensor:
+    """int32 [nseq + 1] offsets of the sequences of ``doc_lengths(S, seed=b)`` for b < B,
+    packed one batch row after another."""
+    lens = [n for b in range(B) for n in doc_lengths(S, b)]
+    return torch.from_numpy(np.concatenate([[0], np.cumsum(lens)]).astype(np.int32))
+
+
 def make_qkv(B: int, H: int, Sq: int, Sk: int, D: int, seed: int = 0,
-             dtype: torch.dtype = torch.bfloat16, q_mul: float = 1.0):
+             dtype: torch.dtype = torch.bfloat16, q_mul: float = 1.0, Hkv: int = 0):
     """Q, K, V drawn i.i.d. N(0,1) on the CPU from one torch generator, in the order
-    q, k, v, then cast to ``dtype``.  Layout [B, H, S, D], contiguous."""
+    q, k, v, then cast to ``dtype``.  Layout [B, H, S, D] ([B, Hkv, Sk, D] for K and V
+    when Hkv is given), contiguous."""
     g = torch.Generator().manual_seed(seed)
+    hk = Hkv or H
     q = torch.randn(B, H, Sq, D, generator=g)
-    k = torch.randn(B, H, Sk, D, generator=g)
-    v = torch.randn(B, H, Sk, D, generator=g)
+    k = torch.randn(B, hk, Sk, D, generator=g)
+    v = torch.randn(B, hk, Sk, D, generator=g)
     if q_mul != 1.0:
         q = q * q_mul
     return q.to(dtype), k.to(dtype), v.to(dtype)

@@ -32,7 +32,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from attn_workloads import (MASK_CAUSAL, MASK_DOC, MASK_WINDOW, WORKLOADS, alibi_slopes,  # noqa: E402
-                            doc_lengths, make_doc_ids, make_fp8_source, make_qkv)
+                            doc_lengths, make_doc_ids, make_fp8_source, make_qkv, varlen_cu_seqlens)
 
 METRIC = "attention fwd TFLOP/s and % of B200 dense BF16/FP8 tensor peak, per config"
 L2_BYTES = 126 * 1024 * 1024
@@ -43,7 +43,7 @@ def visible_pairs(w) -> int:
     """Exact number of visible (i, j) pairs over the whole batch (all b, h)."""
     Sq, Sk = w.Sq, w.Sk
     d = Sk - Sq
-    if w.mask_kind & MASK_DOC:
+    if w.mask_kind & MASK_DOC or w.varlen:
         per_b = []
         for b in range(w.B):
             lens = doc_lengths(Sq, b)
@@ -74,7 +74,7 @@ def algorithmic_flops(w) -> float:
 
 def tile_count_flops(w) -> float:
     """FLOPs counted over the 256x128 tiles the kernel visits (analytic masks only)."""
-    if w.mask_kind & MASK_DOC:
+    if w.mask_kind & MASK_DOC or w.varlen:
         return float("nan")
     nqb = (w.Sq + 255) // 256
     d = w.Sk - w.Sq
@@ -213,8 +213,12 @@ def oracle_sample(w, budget_s: float, seed: int = 0):
     from oracle.attention import attention_fwd, visible_mask
     q, k, v = make_qkv(1, 1, w.Sq, w.Sk, w.D, seed=seed)
     sl = alibi_slopes(w.H)[:1].numpy() if w.alibi else None
-    doc = make_doc_ids(1, w.Sq) if w.doc else None
+    # packed sequences of the document lengths attend exactly as the document mask does
+    doc = make_doc_ids(1, w.Sq) if (w.doc or w.varlen) else None
     doc_np = None if doc is None else doc[0].numpy()
+    if w.varlen:
+        import dataclasses
+        w = dataclasses.replace(w, mask_kind=w.mask_kind | MASK_DOC)
 
     def flops_of(rows):
         vis = 0
@@ -285,7 +289,8 @@ def run_reference(args, w):
 
 
 def workload_config(w):
-    return {"workload": w.note, "B": w.B, "H": w.H, "Sq": w.Sq, "Sk": w.Sk, "D": w.D,
+    return {"workload": w.note, "B": w.B, "H": w.H, "Hkv": w.kv_heads, "Sq": w.Sq, "Sk": w.Sk, "D": w.D,
+            "packed_sequences": w.varlen,
             "mask": {"causal": bool(w.mask_kind & MASK_CAUSAL), "window": w.window,
                      "alibi": w.alibi, "softcap": w.softcap, "document": w.doc},
             "flops": "exact: 4*D per visible (i,j) pair",
@@ -301,32 +306,58 @@ class Case:
     def __init__(self, ta, w, dev, seed):
         self.w, self.ta, self.dev = w, ta, dev
         self.stream = torch.cuda.current_stream(dev)
+        self.cu = None
         if w.fp8:
             self.host = make_fp8_source(w.B, w.H, w.Sq, w.D, seed=seed)
+        elif w.varlen:
+            # B batch rows of S tokens each, packed token-major [T, H, D]
+            cu = varlen_cu_seqlens(w.B, w.Sq)
+            T = int(cu[-1])
+            q, k, v = make_qkv(1, w.H, T, T, w.D, seed=seed, Hkv=w.kv_heads)
+            self.host = tuple(t[0].permute(1, 0, 2).contiguous() for t in (q, k, v))
+            self.cu = cu.to(dev)
+            self.maxlen = int(np.diff(cu.numpy()).max())
         else:
-            self.host = make_qkv(w.B, w.H, w.Sq, w.Sk, w.D, seed=seed)
+            self.host = make_qkv(w.B, w.H, w.Sq, w.Sk, w.D, seed=seed, Hkv=w.kv_heads)
         self.q, self.k, self.v = (t.to(dev).contiguous() for t in self.host)
         sl = alibi_slopes(w.H) if w.alibi else None
         doc = make_doc_ids(w.B, w.Sq) if w.doc else None
         self.sl = None if sl is None else sl.to(dev)
         self.doc = None if doc is None else doc.to(dev)
-        self.o = torch.empty(w.B, w.H, w.Sq, w.D, dtype=torch.bfloat16, device=dev)
-        self.lse = torch.empty(w.B, w.H, w.Sq, dtype=torch.float32, device=dev)
+        if w.varlen:
+            T = self.q.shape[0]
+            self.o = torch.empty(T, w.H, w.D, dtype=torch.bfloat16, device=dev)
+            self.lse = torch.empty(w.H, T, dtype=torch.float32, device=dev)
+        else:
+            self.o = torch.empty(w.B, w.H, w.Sq, w.D, dtype=torch.bfloat16, device=dev)
+            self.lse = torch.empty(w.B, w.H, w.Sq, dtype=torch.float32, device=dev)
         self.launches_per_step = 2 if w.doc else 1
         if w.fp8:
             # e4m3 operands with per-128-row scales, quantised once (the quantiser is timed alone)
             self.q8 = [ta.attn_quantize_e4m3(t, stream=self.stream) for t in (self.q, self.k, self.v)]
 
-    def step(self):
+    def run(self, q, k, v, quantize=False):
+        """The public call a user makes for this workload, on the given inputs."""
         w, ta = self.w, self.ta
         if w.fp8:
-            (q8, qs), (k8, ks), (v8, vs) = self.q8
+            if quantize:
+                a8 = [ta.attn_quantize_e4m3(t, stream=self.stream) for t in (q, k, v)]
+            else:
+                a8 = self.q8
+            (q8, qs), (k8, ks), (v8, vs) = a8
             ta.attn_fwd_fp8(q8, k8, v8, qs, ks, vs, o=self.o, lse=self.lse, scale=w.scale,
                             mask_kind=w.mask_kind, stream=self.stream)
+        elif w.varlen:
+            ta.attn_fwd_varlen(q, k, v, self.cu, self.cu, self.maxlen, self.maxlen, o=self.o, lse=self.lse,
+                               scale=w.scale, mask_kind=w.mask_kind, window=w.window, softcap=w.softcap,
+                               alibi_slopes=self.sl, stream=self.stream)
         else:
-            ta.attn_fwd(self.q, self.k, self.v, o=self.o, lse=self.lse, scale=w.scale, mask_kind=w.mask_kind,
+            ta.attn_fwd(q, k, v, o=self.o, lse=self.lse, scale=w.scale, mask_kind=w.mask_kind,
                         window=w.window, softcap=w.softcap, alibi_slopes=self.sl, doc_ids=self.doc,
                         stream=self.stream)
+
+    def step(self):
+        self.run(self.q, self.k, self.v)
 
     def quantize_ms(self, reps=5):
         ta = self.ta
@@ -369,7 +400,7 @@ def time_launches(step, n, stream, dev, flush=None):
 def compulsory_bytes(w) -> int:
     """Bytes each launch must move at least: Q, K, V read once, O and LSE written once."""
     eb = 1 if w.fp8 else 2
-    qkv = w.B * w.H * (w.Sq + 2 * w.Sk) * w.D * eb
+    qkv = w.B * (w.H * w.Sq + 2 * w.kv_heads * w.Sk) * w.D * eb
     scales = 3 * w.B * w.H * ((w.Sk + 127) // 128) * 4 if w.fp8 else 0
     return qkv + scales + w.B * w.H * w.Sq * (w.D * 2 + 4)
 
@@ -563,13 +594,7 @@ def main():
         q2.copy_(qh, non_blocking=True)
         k2.copy_(kh, non_blocking=True)
         v2.copy_(vh, non_blocking=True)
-        if w.fp8:
-            a8 = [ta.attn_quantize_e4m3(t, stream=stream) for t in (q2, k2, v2)]
-            ta.attn_fwd_fp8(a8[0][0], a8[1][0], a8[2][0], a8[0][1], a8[1][1], a8[2][1], o=case.o, lse=case.lse,
-                            scale=w.scale, mask_kind=w.mask_kind, stream=stream)
-        else:
-            ta.attn_fwd(q2, k2, v2, o=case.o, lse=case.lse, scale=w.scale, mask_kind=w.mask_kind,
-                        window=w.window, softcap=w.softcap, alibi_slopes=case.sl, doc_ids=case.doc, stream=stream)
+        case.run(q2, k2, v2, quantize=True)
         oh.copy_(case.o, non_blocking=True)
         lh.copy_(case.lse, non_blocking=True)
 

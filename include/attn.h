@@ -103,6 +103,45 @@ ATTN_API int attn_fwd(const void* q, const void* k, const void* v, void* o, floa
              const float* alibi_slopes, const int* doc_ids, void* stream);
 
 /*
+ * attn_fwd_gqa — attn_fwd with grouped-query / multi-query heads: H query heads share
+ * H_kv key/value heads (H_kv divides H; query head h reads key/value head h / (H / H_kv);
+ * H_kv = 1 is multi-query attention, H_kv = H is attn_fwd).  Grouped heads: page
+ * "FlashAttention 4: ...", section "Συμβατότητα και τρέχουσα κατάσταση".
+ *   q  bf16 [B,H,Sq,D];  k, v  bf16 [B,H_kv,Sk,D];  o, lse and every other argument as
+ *   attn_fwd (alibi_slopes has H entries, one per query head).
+ */
+ATTN_API int attn_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse,
+                          int B, int H, int H_kv, int Sq, int Sk, int D, float scale,
+                          int mask_kind, int window, float softcap,
+                          const float* alibi_slopes, const int* doc_ids, void* stream);
+
+/*
+ * attn_fwd_varlen — attention over packed variable-length sequences, without padding
+ * (page "FlashAttention 4: ...", section "Συμβατότητα και τρέχουσα κατάσταση").
+ * Sequence s owns query tokens cu_seqlens_q[s] .. cu_seqlens_q[s+1]-1 and key tokens
+ * cu_seqlens_k[s] .. cu_seqlens_k[s+1]-1 and attends only within itself; masks, causal
+ * alignment (bottom-right) and ALiBi positions are per sequence, as if each sequence were
+ * its own batch entry.  Token-major tensors:
+ *   q  bf16 [total_q, H, D];  k, v  bf16 [total_k, H_kv, D]  (device, read)
+ *   o  bf16 [total_q, H, D];  lse  fp32 [H, total_q]         (device, written)
+ *   cu_seqlens_q / cu_seqlens_k  device int32 [nseq + 1], non-decreasing, starting at 0
+ *   max_seqlen_q / max_seqlen_k  upper bounds of the sequence lengths (the work is laid
+ *   out for them); total_q / total_k >= 1 the token counts of the tensors.
+ * mask_kind: CAUSAL and WINDOW (DOC is rejected: the sequences are the documents).  Other
+ * arguments as attn_fwd_gqa.  The offsets live in device memory, so the host cannot check
+ * them: a sequence that leaves its tensor or exceeds a stated maximum is skipped (its
+ * outputs are not written) and ATTN_ERR_INVALID is recorded for attn_get_status.  Key rows
+ * past a sequence's end are masked; their V values are multiplied by 0, so they must be
+ * finite (the tokens of the neighbouring sequence, or TMA zero fill past total_k).
+ */
+ATTN_API int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                             const int* cu_seqlens_q, const int* cu_seqlens_k, int nseq,
+                             int max_seqlen_q, int max_seqlen_k, int total_q, int total_k,
+                             int H, int H_kv, int D, float scale,
+                             int mask_kind, int window, float softcap,
+                             const float* alibi_slopes, void* stream);
+
+/*
  * attn_fwd_noalloc — attn_fwd that allocates no device memory.  (An addition of this
  * library; the method itself has no counterpart for it.)
  * Meant for callers that cannot allocate during a call: code inside a framework whose own
@@ -189,7 +228,8 @@ ATTN_API int attn_fwd_fp8(const void* q8, const void* k8, const void* v8,
 /*
  * attn_get_status — synchronises `stream`, then returns and clears the current device's
  * status word: ATTN_OK, or ATTN_ERR_TIMEOUT if a kernel's bounded wait ran out since the
- * last call (that kernel abandoned its work item and left its outputs undefined), or
+ * last call (that kernel abandoned its work item and left its outputs undefined),
+ * ATTN_ERR_INVALID if attn_fwd_varlen met sequence offsets outside its tensors, or
  * ATTN_ERR_CUDA if the synchronisation itself failed.
  */
 ATTN_API int attn_get_status(void* stream);

@@ -13,7 +13,7 @@ import torch
 from ._lib import (ATTN_ERR_TIMEOUT, ATTN_OK, MASK_CAUSAL, MASK_DOC, MASK_NONE, MASK_WINDOW,
                    AttnError, check, load)
 
-__all__ = ["attn_fwd", "attn_fwd_noalloc", "attn_fwd_with_map", "attn_fwd_fp8", "attn_quantize_e4m3",
+__all__ = ["attn_fwd", "attn_fwd_varlen", "attn_fwd_noalloc", "attn_fwd_with_map", "attn_fwd_fp8", "attn_quantize_e4m3",
            "attn_tile_map_build", "attn_get_status", "attn_shutdown", "tile_map_shape",
            "AttnError", "MASK_NONE", "MASK_CAUSAL", "MASK_WINDOW", "MASK_DOC"]
 
@@ -44,8 +44,9 @@ def _need(t, name, dtype, shape, device):
         raise ValueError(f"{name}: must be contiguous")
 
 
-def _check_qkv(q, k, v, dtype):
-    """q [B,H,Sq,D], k and v [B,H,Sk,D] of ``dtype``, contiguous, on one CUDA device."""
+def _check_qkv(q, k, v, dtype, gqa=False):
+    """q [B,H,Sq,D], k and v [B,H,Sk,D] (with ``gqa``: [B,Hkv,Sk,D], Hkv dividing H) of
+    ``dtype``, contiguous, on one CUDA device."""
     if not isinstance(q, torch.Tensor) or q.dim() != 4:
         raise ValueError("q: expected a 4-d tensor [B, H, Sq, D]")
     if q.device.type != "cuda":
@@ -54,9 +55,15 @@ def _check_qkv(q, k, v, dtype):
     _need(q, "q", dtype, (B, H, Sq, D), q.device)
     if not isinstance(k, torch.Tensor) or k.dim() != 4:
         raise ValueError("k: expected a 4-d tensor [B, H, Sk, D]")
-    Sk = k.shape[2]
-    _need(k, "k", dtype, (B, H, Sk, D), q.device)
-    _need(v, "v", dtype, (B, H, Sk, D), q.device)
+    Hkv, Sk = k.shape[1], k.shape[2]
+    if not gqa and Hkv != H:
+        raise ValueError(f"k: {Hkv} heads, expected {H}")
+    if Hkv < 1 or H % Hkv != 0:
+        raise ValueError(f"k: {Hkv} key/value heads do not divide {H} query heads")
+    _need(k, "k", dtype, (B, Hkv, Sk, D), q.device)
+    _need(v, "v", dtype, (B, Hkv, Sk, D), q.device)
+    if gqa:
+        return B, H, Hkv, Sq, Sk, D
     return B, H, Sq, Sk, D
 
 
@@ -82,17 +89,62 @@ def _out(q, o, lse):
 
 def attn_fwd(q, k, v, o=None, lse=None, scale=None, mask_kind=MASK_NONE, window=0, softcap=0.0,
              alibi_slopes=None, doc_ids=None, stream=None):
-    """BF16 attention forward. q [B,H,Sq,D], k/v [B,H,Sk,D] bf16 contiguous on one device.
+    """BF16 attention forward. q [B,H,Sq,D], k/v [B,Hkv,Sk,D] bf16 contiguous on one device;
+    Hkv < H (dividing it) selects grouped-query heads (attn_fwd_gqa).
     Returns (o bf16 [B,H,Sq,D], lse fp32 [B,H,Sq])."""
     lib = load()
-    B, H, Sq, Sk, D = _check_qkv(q, k, v, torch.bfloat16)
+    B, H, Hkv, Sq, Sk, D = _check_qkv(q, k, v, torch.bfloat16, gqa=True)
     _check_mods(q, H, B, Sk, alibi_slopes, doc_ids)
     o, lse = _out(q, o, lse)
     scale = 1.0 / math.sqrt(D) if scale is None else scale
-    rc = lib.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Sq, Sk, D, float(scale),
-                      int(mask_kind), int(window), float(softcap), _ptr(alibi_slopes), _ptr(doc_ids),
-                      _stream(stream))
-    check(rc, "attn_fwd")
+    if Hkv == H:
+        rc = lib.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Sq, Sk, D, float(scale),
+                          int(mask_kind), int(window), float(softcap), _ptr(alibi_slopes), _ptr(doc_ids),
+                          _stream(stream))
+        check(rc, "attn_fwd")
+    else:
+        rc = lib.attn_fwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Hkv, Sq, Sk, D, float(scale),
+                              int(mask_kind), int(window), float(softcap), _ptr(alibi_slopes), _ptr(doc_ids),
+                              _stream(stream))
+        check(rc, "attn_fwd_gqa")
+    return o, lse
+
+
+def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, o=None, lse=None,
+                    scale=None, mask_kind=MASK_NONE, window=0, softcap=0.0, alibi_slopes=None, stream=None):
+    """Packed variable-length sequences.  q [Tq,H,D], k/v [Tk,Hkv,D] bf16; cu_seqlens_* int32
+    [nseq+1] on the same device.  Returns (o bf16 [Tq,H,D], lse fp32 [H,Tq])."""
+    lib = load()
+    for name, t in (("q", q), ("k", k)):
+        if not isinstance(t, torch.Tensor) or t.dim() != 3 or t.device.type != "cuda":
+            raise ValueError(f"{name}: expected a 3-d CUDA tensor [T, heads, D]")
+    Tq, H, D = q.shape
+    Tk, Hkv = k.shape[0], k.shape[1]
+    if Hkv < 1 or H % Hkv != 0:
+        raise ValueError(f"k: {Hkv} key/value heads do not divide {H} query heads")
+    _need(q, "q", torch.bfloat16, (Tq, H, D), q.device)
+    _need(k, "k", torch.bfloat16, (Tk, Hkv, D), q.device)
+    _need(v, "v", torch.bfloat16, (Tk, Hkv, D), q.device)
+    if not isinstance(cu_seqlens_q, torch.Tensor) or cu_seqlens_q.dim() != 1:
+        raise ValueError("cu_seqlens_q: expected a 1-d int32 tensor [nseq + 1]")
+    nseq = cu_seqlens_q.shape[0] - 1
+    _need(cu_seqlens_q, "cu_seqlens_q", torch.int32, (nseq + 1,), q.device)
+    _need(cu_seqlens_k, "cu_seqlens_k", torch.int32, (nseq + 1,), q.device)
+    _check_mods(q, H, 1, Tk, alibi_slopes, None)
+    if o is None:
+        o = torch.empty(Tq, H, D, dtype=torch.bfloat16, device=q.device)
+    else:
+        _need(o, "o", torch.bfloat16, (Tq, H, D), q.device)
+    if lse is None:
+        lse = torch.empty(H, Tq, dtype=torch.float32, device=q.device)
+    else:
+        _need(lse, "lse", torch.float32, (H, Tq), q.device)
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    rc = lib.attn_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(cu_seqlens_q),
+                             _ptr(cu_seqlens_k), nseq, int(max_seqlen_q), int(max_seqlen_k), Tq, Tk, H, Hkv, D,
+                             float(scale), int(mask_kind), int(window), float(softcap), _ptr(alibi_slopes),
+                             _stream(stream))
+    check(rc, "attn_fwd_varlen")
     return o, lse
 
 

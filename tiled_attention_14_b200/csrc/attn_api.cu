@@ -85,6 +85,19 @@ int check_common(const void* q, const void* k, const void* v, const void* o, con
   return ATTN_OK;
 }
 
+// Packed token-major tensor [T, Hx, D]: map (D, Hx, T), box 64 or 128 columns x 1 head x
+// 128 tokens, so a box lands in shared memory exactly as a batched tile does.
+int encode_map_thd(CUtensorMap* map, const void* ptr, int Hx, int T, int D) {
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Hx), static_cast<cuuint64_t>(T)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(Hx) * D * 2};
+  cuuint32_t box[3] = {64u, 1u, 128u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
 int encode_map(CUtensorMap* map, const void* ptr, bool fp8, int BH, int S, int D) {
   const int eb = fp8 ? 1 : 2;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(S), static_cast<cuuint64_t>(BH)};
@@ -128,7 +141,7 @@ int launch_fwd_d(int dev, const CUtensorMap& tq, const CUtensorMap& tk, const CU
 }
 
 // Fills the parameter block shared by the BF16 and FP8 paths.
-FwdParams make_params(void* o, float* lse, int B, int H, int Sq, int Sk, float scale, int mask_kind,
+FwdParams make_params(void* o, float* lse, int B, int H, int Hkv, int Sq, int Sk, float scale, int mask_kind,
                       int window, float softcap, const float* alibi, const int* doc_ids) {
   FwdParams p;
   std::memset(&p, 0, sizeof(p));
@@ -136,6 +149,8 @@ FwdParams make_params(void* o, float* lse, int B, int H, int Sq, int Sk, float s
   p.lse = lse;
   p.B = B;
   p.H = H;
+  p.Hkv = Hkv;
+  p.group = H / Hkv;
   p.Sq = Sq;
   p.Sk = Sk;
   p.nqb = (Sq + 255) / 256;
@@ -185,11 +200,12 @@ size_t ws_bytes_for_map(int B, int Sq, int Sk) {
 
 // Shared body of attn_fwd / attn_fwd_with_map / attn_fwd_fp8.
 int run_fwd(bool fp8, const void* q, const void* k, const void* v, const float* qs, const float* ks,
-            const float* vs, void* o, float* lse, int B, int H, int Sq, int Sk, int D, float scale,
+            const float* vs, void* o, float* lse, int B, int H, int Hkv, int Sq, int Sk, int D, float scale,
             int mask_kind, int window, float softcap, const float* alibi, const int* doc_ids,
             const int* counts, const uint32_t* entries, cudaStream_t stream) {
   int rc = check_common(q, k, v, o, lse, B, H, Sq, Sk, D, scale, mask_kind, window, softcap, alibi, doc_ids);
   if (rc != ATTN_OK) return rc;
+  if (Hkv <= 0 || H % Hkv != 0) return ATTN_ERR_INVALID;
   if (fp8 && (D != 128 || !qs || !ks || !vs)) return ATTN_ERR_INVALID;
   if ((counts == nullptr) != (entries == nullptr)) return ATTN_ERR_INVALID;
   // the tile-map build launches one grid row per batch entry (grid.y <= 65535)
@@ -197,7 +213,7 @@ int run_fwd(bool fp8, const void* q, const void* k, const void* v, const float* 
   int dev = 0;
   if ((rc = current_device(&dev)) != ATTN_OK) return rc;
 
-  FwdParams p = make_params(o, lse, B, H, Sq, Sk, scale, mask_kind, window, softcap, alibi, doc_ids);
+  FwdParams p = make_params(o, lse, B, H, Hkv, Sq, Sk, scale, mask_kind, window, softcap, alibi, doc_ids);
   if (fp8) {
     p.q_scale = qs;
     p.k_scale = ks;
@@ -206,8 +222,8 @@ int run_fwd(bool fp8, const void* q, const void* k, const void* v, const float* 
     p.nsb_k = (Sk + 127) / 128;
   }
   CUtensorMap tq, tk, tv;
-  if (encode_map(&tq, q, fp8, B * H, Sq, D) != ATTN_OK || encode_map(&tk, k, fp8, B * H, Sk, D) != ATTN_OK ||
-      encode_map(&tv, v, fp8, B * H, Sk, D) != ATTN_OK)
+  if (encode_map(&tq, q, fp8, B * H, Sq, D) != ATTN_OK || encode_map(&tk, k, fp8, B * Hkv, Sk, D) != ATTN_OK ||
+      encode_map(&tv, v, fp8, B * Hkv, Sk, D) != ATTN_OK)
     return ATTN_ERR_CUDA;
 
   void* ws = nullptr;
@@ -282,7 +298,7 @@ int run_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float*
   void* scratch = nullptr;
   if (need_map && (rc = noalloc_scratch(dev, &scratch)) != ATTN_OK) return rc;
 
-  FwdParams p = make_params(o, lse, B, H, Sq, Sk, scale, mask_kind, window, softcap, alibi, doc_ids);
+  FwdParams p = make_params(o, lse, B, H, H, Sq, Sk, scale, mask_kind, window, softcap, alibi, doc_ids);
   CUtensorMap tq, tk, tv;
   if (encode_map(&tq, q, false, B * H, Sq, D) != ATTN_OK || encode_map(&tk, k, false, B * H, Sk, D) != ATTN_OK ||
       encode_map(&tv, v, false, B * H, Sk, D) != ATTN_OK)
@@ -301,6 +317,40 @@ int run_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float*
   return launch_fwd_d<64, false>(dev, tq, tk, tv, p, sc, al, stream);
 }
 
+// Packed variable-length sequences (token-major tensors).  The work items are
+// (sequence, head, 256-row block) up to the longest sequence; blocks past the end of a
+// shorter sequence are empty.  The kernel checks each sequence's bounds against the totals
+// and the maximum lengths and records ATTN_ERR_INVALID (skipping that sequence) if they fail.
+int run_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu_q,
+                   const int* cu_k, int nseq, int max_sq, int max_sk, int total_q, int total_k, int H, int Hkv,
+                   int D, float scale, int mask_kind, int window, float softcap, const float* alibi,
+                   cudaStream_t stream) {
+  if (!cu_q || !cu_k || nseq <= 0) return ATTN_ERR_INVALID;
+  if (total_q <= 0 || total_k <= 0 || max_sq <= 0 || max_sk <= 0) return ATTN_ERR_INVALID;
+  if (max_sq > total_q || max_sk > total_k) return ATTN_ERR_INVALID;
+  if (mask_kind & ATTN_MASK_DOC) return ATTN_ERR_INVALID;   // sequences already separate documents
+  int rc = check_common(q, k, v, o, lse, nseq, H, max_sq, max_sk, D, scale, mask_kind, window, softcap, alibi,
+                        nullptr);
+  if (rc != ATTN_OK) return rc;
+  if (Hkv <= 0 || H % Hkv != 0) return ATTN_ERR_INVALID;
+  if (static_cast<long long>(total_q) * H > 0x7fffffffLL || static_cast<long long>(total_k) * Hkv > 0x7fffffffLL)
+    return ATTN_ERR_INVALID;
+  int dev = 0;
+  if ((rc = current_device(&dev)) != ATTN_OK) return rc;
+  FwdParams p = make_params(o, lse, nseq, H, Hkv, max_sq, max_sk, scale, mask_kind, window, softcap, alibi, nullptr);
+  p.cu_q = cu_q;
+  p.cu_k = cu_k;
+  p.Tq = total_q;
+  p.Tk = total_k;
+  CUtensorMap tq, tk, tv;
+  if (encode_map_thd(&tq, q, H, total_q, D) != ATTN_OK || encode_map_thd(&tk, k, Hkv, total_k, D) != ATTN_OK ||
+      encode_map_thd(&tv, v, Hkv, total_k, D) != ATTN_OK)
+    return ATTN_ERR_CUDA;
+  const bool sc = softcap > 0.f, al = alibi != nullptr;
+  if (D == 128) return launch_fwd_d<128, false>(dev, tq, tk, tv, p, sc, al, stream);
+  return launch_fwd_d<64, false>(dev, tq, tk, tv, p, sc, al, stream);
+}
+
 }  // namespace
 
 extern "C" {
@@ -308,8 +358,24 @@ extern "C" {
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Sq, int Sk,
              int D, float scale, int mask_kind, int window, float softcap, const float* alibi_slopes,
              const int* doc_ids, void* stream) {
-  return run_fwd(false, q, k, v, nullptr, nullptr, nullptr, o, lse, B, H, Sq, Sk, D, scale, mask_kind, window,
+  return run_fwd(false, q, k, v, nullptr, nullptr, nullptr, o, lse, B, H, H, Sq, Sk, D, scale, mask_kind, window,
                  softcap, alibi_slopes, doc_ids, nullptr, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+int attn_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv,
+                 int Sq, int Sk, int D, float scale, int mask_kind, int window, float softcap,
+                 const float* alibi_slopes, const int* doc_ids, void* stream) {
+  return run_fwd(false, q, k, v, nullptr, nullptr, nullptr, o, lse, B, H, H_kv, Sq, Sk, D, scale, mask_kind,
+                 window, softcap, alibi_slopes, doc_ids, nullptr, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu_seqlens_q,
+                    const int* cu_seqlens_k, int nseq, int max_seqlen_q, int max_seqlen_k, int total_q,
+                    int total_k, int H, int H_kv, int D, float scale, int mask_kind, int window, float softcap,
+                    const float* alibi_slopes, void* stream) {
+  return run_fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, nseq, max_seqlen_q, max_seqlen_k, total_q,
+                        total_k, H, H_kv, D, scale, mask_kind, window, softcap, alibi_slopes,
+                        static_cast<cudaStream_t>(stream));
 }
 
 int attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Sq,
@@ -324,7 +390,7 @@ int attn_fwd_with_map(const void* q, const void* k, const void* v, void* o, floa
                       const float* alibi_slopes, const int* doc_ids, const int* counts, const uint32_t* entries,
                       void* stream) {
   if (!counts || !entries) return ATTN_ERR_INVALID;
-  return run_fwd(false, q, k, v, nullptr, nullptr, nullptr, o, lse, B, H, Sq, Sk, D, scale, mask_kind, window,
+  return run_fwd(false, q, k, v, nullptr, nullptr, nullptr, o, lse, B, H, H, Sq, Sk, D, scale, mask_kind, window,
                  softcap, alibi_slopes, doc_ids, counts, entries, static_cast<cudaStream_t>(stream));
 }
 
@@ -334,7 +400,7 @@ int attn_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_
                  void* stream) {
   if (!q_scale || !k_scale || !v_scale) return ATTN_ERR_INVALID;
   if (!aligned16(q_scale) || !aligned16(k_scale) || !aligned16(v_scale)) return ATTN_ERR_INVALID;
-  return run_fwd(true, q8, k8, v8, q_scale, k_scale, v_scale, o, lse, B, H, Sq, Sk, D, scale, mask_kind, window,
+  return run_fwd(true, q8, k8, v8, q_scale, k_scale, v_scale, o, lse, B, H, H, Sq, Sk, D, scale, mask_kind, window,
                  softcap, alibi_slopes, doc_ids, nullptr, nullptr, static_cast<cudaStream_t>(stream));
 }
 

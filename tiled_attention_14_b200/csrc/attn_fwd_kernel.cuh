@@ -78,8 +78,14 @@ __device__ int g_attn_status;
 struct FwdParams {
   __nv_bfloat16* o;
   float* lse;
-  int B, H, Sq, Sk;
-  int nqb, nkt;            // 256-row query blocks, 128-column key tiles
+  int B, H, Sq, Sk;        // packed sequences: Sq, Sk are the longest query / key lengths
+  int Hkv, group;          // key/value heads; query head h reads key/value head h / group
+  int nqb, nkt;            // 256-row query blocks, 128-column key tiles (per sequence)
+  // Packed variable-length sequences (token-major [T, H, D] tensors, LSE [H, Tq]):
+  // sequence s owns tokens cu_q[s] .. cu_q[s+1]-1 (queries) and cu_k[s] .. cu_k[s+1]-1 (keys).
+  const int* cu_q;         // [nseq + 1] or nullptr (batched [B, H, S, D] tensors)
+  const int* cu_k;
+  int Tq, Tk;              // total query / key tokens (LSE layout [H, Tq])
   int mask_kind, window;   // window already clamped to <= Sq + Sk
   float scale_log2;        // scale * log2(e)
   float sc_in, sc_out;     // soft-capping: x = s * sc_in, t = tanh(x) * sc_out (log2 units)
@@ -214,14 +220,17 @@ __device__ __forceinline__ bool drain_bounded(uint32_t bar, uint32_t parity,
 // ---------------------------------------------------------------------------------------
 struct Item {
   int b, h, bh, qb;
+  int kvbh;       // key/value head row of the K/V tensors (b * Hkv + h / group)
+  int sq, sk;     // query and key lengths of this item's sequence
+  int q_off, k_off;  // first query / key token of the sequence (packed layout; else 0)
   int n;          // number of key tiles visited
   int kt_lo;      // analytic: first key tile
   const uint32_t* entries;  // map: entry list (nullptr for analytic)
 };
 
-__device__ __forceinline__ int hi_key(const FwdParams& p, int ip) {  // last visible key of row i'
-  int h = (p.mask_kind & 1) ? ip : ((p.mask_kind & 2) ? ip + p.window - 1 : p.Sk - 1);
-  return min(h, p.Sk - 1);
+__device__ __forceinline__ int hi_key(const FwdParams& p, int sk, int ip) {  // last visible key of row i'
+  int h = (p.mask_kind & 1) ? ip : ((p.mask_kind & 2) ? ip + p.window - 1 : sk - 1);
+  return min(h, sk - 1);
 }
 __device__ __forceinline__ int lo_key(const FwdParams& p, int ip) {  // first visible key (unclipped)
   return (p.mask_kind & 2) ? ip - p.window + 1 : 0;
@@ -232,7 +241,7 @@ __device__ __forceinline__ int lo_key(const FwdParams& p, int ip) {  // first vi
 // all heads; otherwise the order is head-major (the K/V of one head stay hot in L2).
 __device__ __forceinline__ Item make_item(const FwdParams& p, int w) {
   Item it;
-  const int BH = p.B * p.H;
+  const int BH = p.B * p.H;   // packed sequences: B is the number of sequences
   if (p.lpt_qb_major) {
     it.qb = p.nqb - 1 - w / BH;
     it.bh = w % BH;
@@ -242,6 +251,24 @@ __device__ __forceinline__ Item make_item(const FwdParams& p, int w) {
   }
   it.b = it.bh / p.H;
   it.h = it.bh % p.H;
+  it.kvbh = it.b * p.Hkv + it.h / p.group;
+  if (p.cu_q != nullptr) {
+    it.q_off = __ldg(p.cu_q + it.b);
+    it.sq = __ldg(p.cu_q + it.b + 1) - it.q_off;
+    it.k_off = __ldg(p.cu_k + it.b);
+    it.sk = __ldg(p.cu_k + it.b + 1) - it.k_off;
+    // Offsets come from device memory: a sequence outside the tensors or longer than the
+    // stated maximum is skipped (nothing loaded or stored) and reported.
+    if (it.q_off < 0 || it.sq < 0 || it.sq > p.Sq || it.q_off > p.Tq - it.sq || it.k_off < 0 || it.sk < 0 ||
+        it.sk > p.Sk || it.k_off > p.Tk - it.sk) {
+      if (it.qb == 0 && it.h == 0) atomicCAS(&g_attn_status, 0, -1 /* ATTN_ERR_INVALID */);
+      it.q_off = it.k_off = it.sq = it.sk = 0;
+    }
+  } else {
+    it.q_off = it.k_off = 0;
+    it.sq = p.Sq;
+    it.sk = p.Sk;
+  }
   it.entries = nullptr;
   it.kt_lo = 0;
   if (p.map_counts != nullptr) {
@@ -249,13 +276,14 @@ __device__ __forceinline__ Item make_item(const FwdParams& p, int w) {
     it.entries = p.map_entries + (static_cast<size_t>(it.b) * p.nqb + it.qb) * p.nkt;
     return it;
   }
-  const int d = p.Sk - p.Sq;
+  const int d = it.sk - it.sq;
   int A = it.qb * 256 + d;
-  const int Bm = min(it.qb * 256 + 255, p.Sq - 1) + d;
+  const int Bm = min(it.qb * 256 + 255, it.sq - 1) + d;
   if (p.mask_kind & 1) A = max(A, 0);
   const int klo = max(0, lo_key(p, A));
-  const int khi = hi_key(p, Bm);
-  if (((p.mask_kind & 1) && Bm < 0) || khi < klo) {
+  const int khi = hi_key(p, it.sk, Bm);
+  // a block past the end of its sequence (packed layout) or with no visible key
+  if (it.qb * 256 >= it.sq || ((p.mask_kind & 1) && Bm < 0) || khi < klo) {
     it.n = 0;
     return it;
   }
@@ -278,16 +306,16 @@ __device__ __forceinline__ int tile_kt(const Item& it, int i) {
 __device__ __forceinline__ int tile_class(const FwdParams& p, const Item& it, int i, int g, int kt) {
   if (it.entries) return static_cast<int>((__ldg(it.entries + i) >> (24 + 2 * g)) & 3u);
   const int r0 = it.qb * 256 + 128 * g;
-  if (r0 >= p.Sq) return 0;
-  const int r1 = min(r0 + 127, p.Sq - 1);
-  const int d = p.Sk - p.Sq;
+  if (r0 >= it.sq) return 0;
+  const int r1 = min(r0 + 127, it.sq - 1);
+  const int d = it.sk - it.sq;
   const int a = r0 + d, bb = r1 + d;
-  const int c0 = kt * 128, c1 = c0 + 127, c1v = min(c1, p.Sk - 1);
+  const int c0 = kt * 128, c1 = c0 + 127, c1v = min(c1, it.sk - 1);
   const bool causal = p.mask_kind & 1, win = p.mask_kind & 2;
   const int i1 = causal ? c0 : (win ? c0 - p.window + 1 : INT_MIN);
   const int i2 = win ? c1v + p.window - 1 : INT_MAX;
   if (max(a, i1) > min(bb, i2)) return 0;
-  const bool full = (c1 <= p.Sk - 1) && (!win || bb - p.window + 1 <= c0) &&
+  const bool full = (c1 <= it.sk - 1) && (!win || bb - p.window + 1 <= c0) &&
                     (causal ? (a >= c1) : (!win || a + p.window - 1 >= c1));
   return full ? 2 : 1;
 }
@@ -308,7 +336,7 @@ __device__ __forceinline__ void softmax_tile(const FwdParams& p, const Item& it,
       float pv_log2 = 0.f;         // FP8: log2 of the V block's scale relative to v_norm
       float inv_pvf = 1.f;         // and the inverse of that factor
       if constexpr (FP8) {
-        const size_t kb = static_cast<size_t>(it.bh) * p.nsb_k + kt;
+        const size_t kb = static_cast<size_t>(it.kvbh) * p.nsb_k + kt;
         const float sqk = sq_scale * __ldg(p.k_scale + kb);
         sc *= sqk;
         sc_in *= sqk;
@@ -537,6 +565,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   if (warp == kLoadWarp) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
+      const bool varlen = p.cu_q != nullptr;
       const uint64_t pol_kv = policy_evict_last();
       const uint64_t pol_q = policy_evict_first();
       uint32_t lidx = 0;     // ring loads issued (K and V alternate)
@@ -556,9 +585,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             break;
           }
           mbar_expect_tx(BAR(B_QFULL + g), C::TILE_BYTES);
+          // batched tensors: map (D, S, B*H), coordinates (x, row, b*H+h); packed sequences:
+          // map (D, H, T), coordinates (x, h, token)
+          const int qrow = it.qb * 256 + 128 * g;
+          const int qc1 = varlen ? it.h : qrow, qc2 = varlen ? it.q_off + qrow : it.bh;
           for (int pn = 0; pn < C::NPANEL; ++pn)
             tma_load_3d(sbase + C::OFF_Q + g * C::TILE_BYTES + pn * C::PANEL_BYTES, &tm_q,
-                        BAR(B_QFULL + g), pn * C::PANEL_COLS, it.qb * 256 + 128 * g, it.bh, pol_q);
+                        BAR(B_QFULL + g), pn * C::PANEL_COLS, qc1, qc2, pol_q);
           ++q_issued[g];
         }
         if (!ok) break;
@@ -573,9 +606,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             mbar_expect_tx(BAR(B_KVFULL + slot), C::TILE_BYTES);
             const CUtensorMap* tm = kv ? &tm_v : &tm_k;
+            const int kc1 = varlen ? it.kvbh : kt * 128, kc2 = varlen ? it.k_off + kt * 128 : it.kvbh;
             for (int pn = 0; pn < C::NPANEL; ++pn)
               tma_load_3d(sbase + C::OFF_KV + slot * C::TILE_BYTES + pn * C::PANEL_BYTES, tm,
-                          BAR(B_KVFULL + slot), pn * C::PANEL_COLS, kt * 128, it.bh, pol_kv);
+                          BAR(B_KVFULL + slot), pn * C::PANEL_COLS, kc1, kc2, pol_kv);
             ++lidx;
           }
         }
@@ -696,10 +730,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const int w = sched_pos(r, cta, G);
       if (w >= p.num_items) break;
       const Item it = make_item(p, w);
-      const int row = it.qb * 256 + 128 * g + rloc;  // query row
-      const int ip = row + (p.Sk - p.Sq);            // bottom-right aligned position
+      const int row = it.qb * 256 + 128 * g + rloc;  // query row within its sequence
+      const int ip = row + (it.sk - it.sq);          // bottom-right aligned position
       int jlo_row = lo_key(p, ip);
-      int jhi_row = hi_key(p, ip);
+      int jhi_row = hi_key(p, it.sk, ip);
       const int doc_row = (has_doc && row < p.Sq) ? __ldg(p.doc + static_cast<size_t>(it.b) * p.Sk + row) : 0;
       bool doc_elem = has_doc;   // per-element document test needed on PARTIAL tiles
       if (has_doc && p.doc_sorted != nullptr && __ldg(p.doc_sorted + it.b) != 0) {
@@ -723,7 +757,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       if constexpr (FP8) {
         const size_t qbase = static_cast<size_t>(it.bh) * p.nsb_q;
         sq_scale = __ldg(p.q_scale + qbase + min(2 * it.qb + g, p.nsb_q - 1));
-        const size_t vbase = static_cast<size_t>(it.bh) * p.nsb_k;
+        const size_t vbase = static_cast<size_t>(it.kvbh) * p.nsb_k;
         float vm = 0.f;
         for (int sb = 0; sb < p.nsb_k; ++sb) vm = fmaxf(vm, __ldg(p.v_scale + vbase + sb));
         v_norm = vm > 0.f ? vm : 1.f;
@@ -765,7 +799,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tc_fence_after();
       }
       const float inv_l = (l_run > 0.f) ? (v_norm / l_run) : 0.f;
-      __nv_bfloat16* orow = p.o + (static_cast<size_t>(it.bh) * p.Sq + row) * D;
+      // batched: O [B, H, Sq, D], LSE [B, H, Sq]; packed: O [Tq, H, D], LSE [H, Tq]
+      const bool varlen = p.cu_q != nullptr;
+      const size_t orow_idx = varlen ? static_cast<size_t>(it.q_off + row) * p.H + it.h
+                                     : static_cast<size_t>(it.bh) * p.Sq + row;
+      const size_t lse_idx = varlen ? static_cast<size_t>(it.h) * p.Tq + it.q_off + row
+                                    : static_cast<size_t>(it.bh) * p.Sq + row;
+      __nv_bfloat16* orow = p.o + orow_idx * D;
 #pragma unroll
       for (int ch = 0; ch < D / 32; ++ch) {
         uint32_t o[32];
@@ -779,15 +819,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
         for (int c = 0; c < 16; ++c)
           wv[c] = pack_bf16x2(__uint_as_float(o[2 * c]) * inv_l, __uint_as_float(o[2 * c + 1]) * inv_l);
-        if (row < p.Sq) {
+        if (row < it.sq) {
           uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
 #pragma unroll
           for (int v = 0; v < 4; ++v) __stcs(dst + v, make_uint4(wv[4 * v], wv[4 * v + 1], wv[4 * v + 2], wv[4 * v + 3]));
         }
       }
-      if (row < p.Sq) {
+      if (row < it.sq) {
         const float lse = (l_run > 0.f) ? (m_run + lg2_approx(l_run)) * kLn2 : kNegInf;
-        p.lse[static_cast<size_t>(it.bh) * p.Sq + row] = lse;
+        p.lse[lse_idx] = lse;
       }
       tcount += it.n;
     }
