@@ -168,6 +168,29 @@ ATTN_API int attn_fwd_noalloc(const void* q, const void* k, const void* v, void*
                               const float* alibi_slopes, const int* doc_ids, void* stream);
 
 /*
+ * attn_bwd — attention backward: dQ, dK, dV of the forward above (same arguments, score_mod
+ * and masks; grouped-query heads as attn_fwd_gqa) from the forward's inputs, its output O
+ * and log-sum-exp LSE, and the output gradient dO.  The pages compare FA4's backward with
+ * cuDNN's and note that block-sparse backward runs are not deterministic (page "PyTorch's
+ * FlexAttention mit FlashAttention-4 ist ein Game-Changer", sections "Leistung und
+ * Validierung" and "Aktuelle Einschränkungen"); this one is: no floating-point atomics, a
+ * fixed accumulation order, bitwise identical results run to run.  ALiBi slopes get no
+ * gradient (captured tensors get none, same section).
+ *   q, o, dout  bf16 [B,H,Sq,D];  k, v  bf16 [B,H_kv,Sk,D];  lse  fp32 [B,H,Sq] (natural log,
+ *   -inf for rows that saw no key)                                (device, read)
+ *   dq  bf16 [B,H,Sq,D];  dk, dv  bf16 [B,H_kv,Sk,D]              (device, written)
+ * dK and dV of a key/value head sum over the query heads that share it.  Internally fp32:
+ * P and dS are rounded to bf16 as tensor-core operands.  Three launches on `stream` (row
+ * sums of dO*O and log2-scaled LSE into a stream-ordered workspace, then the dK/dV kernel,
+ * then the dQ kernel).  Other arguments and errors as attn_fwd_gqa.
+ */
+ATTN_API int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                      const float* lse, void* dq, void* dk, void* dv,
+                      int B, int H, int H_kv, int Sq, int Sk, int D, float scale,
+                      int mask_kind, int window, float softcap,
+                      const float* alibi_slopes, const int* doc_ids, void* stream);
+
+/*
  * attn_tile_map_build — classify every (256-row query block, 128-column key tile) pair
  * as EMPTY, PARTIAL or FULL under the mask and list the non-empty key tiles.
  *   counts   device int32 [B, ceil(Sq/256)]               (written)

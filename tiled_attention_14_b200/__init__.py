@@ -13,7 +13,7 @@ import torch
 from ._lib import (ATTN_ERR_TIMEOUT, ATTN_OK, MASK_CAUSAL, MASK_DOC, MASK_NONE, MASK_WINDOW,
                    AttnError, check, load)
 
-__all__ = ["attn_fwd", "attn_fwd_varlen", "attn_fwd_noalloc", "attn_fwd_with_map", "attn_fwd_fp8", "attn_quantize_e4m3",
+__all__ = ["attn_fwd", "attn_bwd", "attn_fwd_varlen", "attn_fwd_noalloc", "attn_fwd_with_map", "attn_fwd_fp8", "attn_quantize_e4m3",
            "attn_tile_map_build", "attn_get_status", "attn_shutdown", "tile_map_shape",
            "AttnError", "MASK_NONE", "MASK_CAUSAL", "MASK_WINDOW", "MASK_DOC"]
 
@@ -108,6 +108,32 @@ def attn_fwd(q, k, v, o=None, lse=None, scale=None, mask_kind=MASK_NONE, window=
                               _stream(stream))
         check(rc, "attn_fwd_gqa")
     return o, lse
+
+
+def attn_bwd(q, k, v, o, lse, dout, dq=None, dk=None, dv=None, scale=None, mask_kind=MASK_NONE, window=0,
+             softcap=0.0, alibi_slopes=None, doc_ids=None, stream=None):
+    """Attention backward.  q, o, dout [B,H,Sq,D] bf16, k/v [B,Hkv,Sk,D] bf16, lse fp32
+    [B,H,Sq] from the forward.  Returns (dq [B,H,Sq,D], dk [B,Hkv,Sk,D], dv [B,Hkv,Sk,D])."""
+    lib = load()
+    B, H, Hkv, Sq, Sk, D = _check_qkv(q, k, v, torch.bfloat16, gqa=True)
+    _check_mods(q, H, B, Sk, alibi_slopes, doc_ids)
+    _need(o, "o", torch.bfloat16, (B, H, Sq, D), q.device)
+    _need(dout, "dout", torch.bfloat16, (B, H, Sq, D), q.device)
+    _need(lse, "lse", torch.float32, (B, H, Sq), q.device)
+    outs = []
+    for name, t, shape in (("dq", dq, (B, H, Sq, D)), ("dk", dk, (B, Hkv, Sk, D)), ("dv", dv, (B, Hkv, Sk, D))):
+        if t is None:
+            t = torch.empty(shape, dtype=torch.bfloat16, device=q.device)
+        else:
+            _need(t, name, torch.bfloat16, shape, q.device)
+        outs.append(t)
+    dq, dk, dv = outs
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    rc = lib.attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
+                      B, H, Hkv, Sq, Sk, D, float(scale), int(mask_kind), int(window), float(softcap),
+                      _ptr(alibi_slopes), _ptr(doc_ids), _stream(stream))
+    check(rc, "attn_bwd")
+    return dq, dk, dv
 
 
 def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, o=None, lse=None,

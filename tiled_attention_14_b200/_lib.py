@@ -30,6 +30,7 @@ SIGNATURES = {
     "attn_fwd_gqa": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _F, _P, _P, _P]),
     "attn_fwd_varlen": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _F,
                              _P, _P]),
+    "attn_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _F, _P, _P, _P]),
     "attn_tile_map_build": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P]),
     "attn_fwd_with_map": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _F, _P, _P, _P, _P, _P]),
     "attn_quantize_e4m3": (_I, [_P, _P, _P, _I, _I, _I, _I, _P]),

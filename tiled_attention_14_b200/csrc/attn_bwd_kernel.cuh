@@ -1,0 +1,860 @@
+// attn_bwd_kernel.cuh — fused attention backward for sm_100a (B200).
+//
+// What it computes: the gradients dQ, dK, dV of the attention forward (same score_mod and
+// masks, grouped-query heads included) from Q, K, V, O, dO and the forward's per-row
+// log-sum-exp, so that neither P nor dP ever reaches HBM.  The pages compare FA4's
+// backward passes with cuDNN's and warn that block-sparse backward runs are not
+// deterministic (page "PyTorch's FlexAttention mit FlashAttention-4 ist ein Game-Changer",
+// sections "Leistung und Validierung" and "Aktuelle Einschränkungen"); the page
+// "FlashAttention 4: ..." lists the backward among FA4's missing parts (section "Κύρια
+// Συμπεράσματα").  With t = score_mod(scale * q.k) and P = exp(t - LSE):
+//     dV = P^T dO,  dP = dO V^T,  dS = P * (dP - Dv) * dt/ds,  Dv_i = sum_d dO_id O_id,
+//     dQ = scale * dS K,  dK = scale * dS^T Q.
+//
+// Deterministic by construction: no floating-point atomics.  Three launches:
+//   attn_bwd_prep_kernel   Dv and LSE * log2(e) per query row, padded to 128-row tiles
+//                          (plus a "document ids sorted" flag per batch row)
+//   attn_bwd_dkdv_kernel   one work item = one 128-key tile of one key/value head; it walks
+//                          every (query head of the group, 128-row query tile) that sees the
+//                          tile, accumulating dV and dK in tensor memory in a fixed order
+//   attn_bwd_dq_kernel     one work item = one 128-row query tile of one head; it walks the
+//                          visible key tiles, accumulating dQ in tensor memory
+// dQ is computed apart from dK/dV (recomputing S and dP) instead of being summed across
+// CTAs, which is what keeps the result bit-reproducible.
+//
+// Each kernel: 6 warps — warps 0-3 compute (one thread per TMEM lane = one row of the
+// 128-row tile), warp 4 issues the TMA loads, one thread of warp 5 issues the MMAs.
+// Tensor memory, dK/dV kernel: S^T | dP^T | dV | dK (P^T and dS^T in bf16 over the first
+// columns of S^T and dP^T); dQ kernel: S | dP | dQ (dS over dP).  Every wait is bounded as
+// in the forward kernel.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "attn_fwd_kernel.cuh"
+
+namespace attn {
+
+constexpr int kBwdThreads = 192;
+constexpr int kBwdLoadWarp = 4;
+constexpr int kBwdMmaWarp = 5;
+
+struct BwdParams {
+  __nv_bfloat16* dq;
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+  const float* lse2;       // [B*H, Sq_pad]: LSE * log2(e); +inf for rows without keys and padding
+  const float* dvec;       // [B*H, Sq_pad]: sum_d dO * O; 0 for padding
+  int B, H, Hkv, group, Sq, Sk, Sq_pad;
+  int nqt, nkt;            // 128-row query tiles, 128-key tiles
+  int mask_kind, window;
+  float scale;             // scale of the scores (dQ and dK are multiplied by it at the end)
+  float scale_log2;        // scale * log2(e)
+  float sc_in, sc_out;     // soft-capping: th = tanh(s * sc_in), t = th * sc_out (log2 units)
+  const float* alibi;      // [H] or nullptr
+  const int* doc;          // [B, Sk] or nullptr
+  const int* doc_sorted;   // [B] flags (from the prep kernel) or nullptr
+  int num_items;
+  int lpt;                 // causal: longest items first
+  unsigned long long timeout_ns;
+};
+
+template <int D>
+struct BwdCfg {
+  static constexpr int TILE_BYTES = 128 * D * 2;         // one 128-row bf16 tile
+  static constexpr int PANEL_BYTES = 128 * 128;
+  static constexpr int NPANEL = D / 64;
+  static constexpr int NST = 2;                          // streamed-tile ring depth
+  // dK/dV kernel: K | V | NST x (Q | dO) | NST x (lse2 | dvec) ; dQ kernel: Q | dO | NST x (K | V)
+  static constexpr int OFF_A = 0;                        // K (dkdv) or Q (dq)
+  static constexpr int OFF_B = TILE_BYTES;               // V (dkdv) or dO (dq)
+  static constexpr int OFF_RING = 2 * TILE_BYTES;        // stage s: [OFF_RING + s*2*TILE, +TILE)
+  static constexpr int OFF_ROWS = OFF_RING + NST * 2 * TILE_BYTES;   // NST x 1 KB (lse2, dvec)
+  static constexpr int OFF_BAR = OFF_ROWS + NST * 1024;
+  static constexpr int NBAR = 16;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t T_S = 0, T_DP = 128, T_ACC0 = 256, T_ACC1 = 256 + D;
+  static constexpr uint32_t IDESC_SS = make_idesc(1u, 128, 128, false);   // 128x128, both K-major
+  static constexpr uint32_t IDESC_TS = make_idesc(1u, 128, D, true);      // A from TMEM, B MN-major
+};
+
+// ---------------------------------------------------------------------------------------
+// preparation: Dv = rowsum(dO * O), LSE in log2 units, padded to whole 128-row tiles
+// ---------------------------------------------------------------------------------------
+constexpr int kPrepThreads = 256;   // 8 warps, one query row per warp at a time
+
+template <int D>
+__global__ void __launch_bounds__(kPrepThreads)
+attn_bwd_prep_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
+                     const float* __restrict__ lse, float* __restrict__ lse2, float* __restrict__ dvec,
+                     int Sq, int Sq_pad, long long rows_total) {
+  const int lane = threadIdx.x & 31;
+  const long long warp_g = (static_cast<long long>(blockIdx.x) * kPrepThreads + threadIdx.x) >> 5;
+  const long long nwarps = (static_cast<long long>(gridDim.x) * kPrepThreads) >> 5;
+  for (long long r = warp_g; r < rows_total; r += nwarps) {   // r over (bh, row < Sq_pad)
+    const long long bh = r / Sq_pad;
+    const int row = static_cast<int>(r - bh * Sq_pad);
+    float dsum = 0.f, l2 = __builtin_huge_valf();
+    if (row < Sq) {
+      const size_t base = (static_cast<size_t>(bh) * Sq + row) * D;
+      constexpr int PER = D / 32;   // elements per lane (2 or 4)
+      if constexpr (PER == 4) {
+        const uint2 a = *reinterpret_cast<const uint2*>(o + base + lane * 4);
+        const uint2 b = *reinterpret_cast<const uint2*>(dout + base + lane * 4);
+        const float2 a0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&a.x));
+        const float2 a1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&a.y));
+        const float2 b0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&b.x));
+        const float2 b1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&b.y));
+        dsum = a0.x * b0.x + a0.y * b0.y + a1.x * b1.x + a1.y * b1.y;
+      } else {
+        const uint32_t a = *reinterpret_cast<const uint32_t*>(o + base + lane * 2);
+        const uint32_t b = *reinterpret_cast<const uint32_t*>(dout + base + lane * 2);
+        const float2 a0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&a));
+        const float2 b0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&b));
+        dsum = a0.x * b0.x + a0.y * b0.y;
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, off);
+      const float l = lse[static_cast<size_t>(bh) * Sq + row];
+      l2 = (l == kNegInf) ? __builtin_huge_valf() : l * kLog2e;
+    }
+    if (lane == 0) {
+      lse2[r] = l2;
+      dvec[r] = dsum;
+    }
+  }
+}
+
+// One CTA per batch row: 1 if doc[b, :] is non-decreasing.
+constexpr int kSortedThreads = 256;
+__global__ void __launch_bounds__(kSortedThreads)
+attn_doc_sorted_kernel(const int* __restrict__ doc, int S, int* __restrict__ flags) {
+  const int* d = doc + static_cast<size_t>(blockIdx.x) * S;
+  int ok = 1;
+  for (int i = threadIdx.x; i + 1 < S; i += kSortedThreads) ok &= (__ldg(d + i) <= __ldg(d + i + 1)) ? 1 : 0;
+  ok = __syncthreads_and(ok);
+  if (threadIdx.x == 0) flags[blockIdx.x] = ok;
+}
+
+// ---------------------------------------------------------------------------------------
+// shared helpers
+// ---------------------------------------------------------------------------------------
+// First and last key (or query) position of the document run that contains position x, for
+// non-decreasing ids (two binary searches).
+__device__ __forceinline__ int2 doc_run(const int* drow, int S, int x) {
+  const int id = __ldg(drow + x);
+  int lo = 0, hi = x;
+  while (lo < hi) { const int mid = (lo + hi) >> 1; if (__ldg(drow + mid) < id) lo = mid + 1; else hi = mid; }
+  const int first = lo;
+  lo = x + 1;
+  hi = S;
+  while (lo < hi) { const int mid = (lo + hi) >> 1; if (__ldg(drow + mid) <= id) lo = mid + 1; else hi = mid; }
+  return make_int2(first, lo - 1);
+}
+
+// Query rows (bottom-right aligned: i' = i + Sk - Sq) that may see key j under the
+// interval masks: [first, last] (unclipped).
+__device__ __forceinline__ int2 rows_seeing_key(const BwdParams& p, int j) {
+  const int d = p.Sk - p.Sq;
+  int lo = INT_MIN / 2, hi = INT_MAX / 2;
+  if (p.mask_kind & 1) lo = j - d;
+  if (p.mask_kind & 2) {
+    hi = j - d + p.window - 1;
+    if (!(p.mask_kind & 1)) lo = j - d - p.window + 1;
+  }
+  return make_int2(lo, hi);
+}
+// Keys that query row i may see under the interval masks: [first, last] (unclipped).
+__device__ __forceinline__ int2 keys_seen_by_row(const BwdParams& p, int i) {
+  const int ip = i + p.Sk - p.Sq;
+  int lo = 0, hi = p.Sk - 1;
+  if (p.mask_kind & 1) hi = ip;
+  if (p.mask_kind & 2) {
+    lo = ip - p.window + 1;
+    if (!(p.mask_kind & 1)) hi = ip + p.window - 1;
+  }
+  return make_int2(lo, hi);
+}
+
+// 128-bit mask of the visible columns clo..chi (relative to the tile, may be out of 0..127).
+__device__ __forceinline__ void interval_mask(int clo, int chi, uint32_t (&vm)[4]) {
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    const int lo = min(max(clo - 32 * w, 0), 32), hi = min(max(chi + 1 - 32 * w, 0), 32);
+    const uint32_t below_hi = hi >= 32 ? 0xffffffffu : ((1u << hi) - 1u);
+    const uint32_t below_lo = lo >= 32 ? 0xffffffffu : ((1u << lo) - 1u);
+    vm[w] = below_hi & ~below_lo;
+  }
+}
+
+// score_mod in log2 units for one raw score s at relative position (j - i'):
+// returns t and writes dt/ds / scale (1 without soft-capping) to *fp.
+template <bool SOFTCAP, bool ALIBI>
+__device__ __forceinline__ float bwd_modify(const BwdParams& p, float s, float slope_l2, float rel, float* fp) {
+  float t;
+  if constexpr (SOFTCAP) {
+    const float th = tanh_approx(s * p.sc_in);
+    t = th * p.sc_out;
+    *fp = fmaf(-th, th, 1.f);
+  } else {
+    t = s * p.scale_log2;
+    *fp = 1.f;
+  }
+  if constexpr (ALIBI) t = fmaf(slope_l2, rel, t);
+  return t;
+}
+
+// ---------------------------------------------------------------------------------------
+// dK / dV kernel
+// ---------------------------------------------------------------------------------------
+struct KvItem {
+  int b, kvh, nt;      // batch, key/value head, key tile
+  int m_lo, m_hi;      // query tiles visited: m_lo .. m_hi (per query head of the group)
+  int n;               // steps = group * (m_hi - m_lo + 1), or 0
+};
+
+__device__ __forceinline__ KvItem make_kv_item(const BwdParams& p, int w) {
+  KvItem it;
+  const int BHkv = p.B * p.Hkv;
+  int bkv;
+  if (p.lpt) {   // causal: the first key tiles are seen by the most query tiles
+    it.nt = w / BHkv;
+    bkv = w % BHkv;
+  } else {
+    bkv = w / p.nkt;
+    it.nt = w % p.nkt;
+  }
+  it.b = bkv / p.Hkv;
+  it.kvh = bkv % p.Hkv;
+  const int j0 = it.nt * 128, j1 = min(j0 + 127, p.Sk - 1);
+  int r0 = max(rows_seeing_key(p, j0).x, 0);
+  int r1 = min(rows_seeing_key(p, j1).y, p.Sq - 1);
+  if (p.doc != nullptr && p.doc_sorted != nullptr && __ldg(p.doc_sorted + it.b)) {
+    const int* drow = p.doc + static_cast<size_t>(it.b) * p.Sk;
+    r0 = max(r0, doc_run(drow, p.Sk, j0).x);
+    r1 = min(r1, doc_run(drow, p.Sk, j1).y);
+  }
+  if (r1 < r0) {
+    it.m_lo = 0;
+    it.m_hi = -1;
+    it.n = 0;
+    return it;
+  }
+  it.m_lo = r0 / 128;
+  it.m_hi = r1 / 128;
+  it.n = p.group * (it.m_hi - it.m_lo + 1);
+  return it;
+}
+
+template <int D, bool SOFTCAP, bool ALIBI>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                     const BwdParams p) {
+  using C = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* sptr = smem_raw + (sbase - raw);
+  auto BAR = [&](int i) -> uint32_t { return sbase + C::OFF_BAR + 8 * i; };
+  // barriers
+  constexpr int B_KVFULL = 0, B_KVEMPTY = 1, B_QFULL = 2, B_QEMPTY = 2 + C::NST, B_SFULL = 2 + 2 * C::NST,
+                B_PFULL = B_SFULL + 1, B_DONE = B_PFULL + 1, B_DRAIN = B_DONE + 1;
+  static_assert(B_DRAIN < C::NBAR, "barrier count");
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sptr + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sptr + C::OFF_MISC + 4);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = gridDim.x, cta = blockIdx.x;
+  const unsigned long long tmo = p.timeout_ns;
+
+  if (threadIdx.x == 0) {
+    mbar_init(BAR(B_KVFULL), 1);
+    mbar_init(BAR(B_KVEMPTY), 1);
+    for (int s = 0; s < C::NST; ++s) {
+      mbar_init(BAR(B_QFULL + s), 1);
+      mbar_init(BAR(B_QEMPTY + s), 1);
+    }
+    mbar_init(BAR(B_SFULL), 1);
+    mbar_init(BAR(B_PFULL), 128);
+    mbar_init(BAR(B_DONE), 1);
+    mbar_init(BAR(B_DRAIN), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kBwdMmaWarp) {
+    tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == kBwdLoadWarp && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_do);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_holder;
+
+  if (warp == kBwdLoadWarp) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const uint64_t pol_last = policy_evict_last();
+      uint32_t items = 0, lidx = 0;
+      bool ok = true;
+      for (int r = 0; ok; ++r) {
+        const int w = sched_pos(r, cta, G);
+        if (w >= p.num_items) break;
+        const KvItem it = make_kv_item(p, w);
+        if (it.n == 0) continue;
+        // K and V of this item, once the previous item's last MMAs have read them
+        if (items > 0 && !wait_bounded(BAR(B_KVEMPTY), (items - 1) & 1, abort_flag, tmo)) break;
+        mbar_expect_tx(BAR(B_KVFULL), 2 * C::TILE_BYTES);
+        const int kvrow = it.b * p.Hkv + it.kvh;
+        for (int pn = 0; pn < C::NPANEL; ++pn) {
+          tma_load_3d(sbase + C::OFF_A + pn * C::PANEL_BYTES, &tm_k, BAR(B_KVFULL), pn * 64, it.nt * 128, kvrow,
+                      pol_last);
+          tma_load_3d(sbase + C::OFF_B + pn * C::PANEL_BYTES, &tm_v, BAR(B_KVFULL), pn * 64, it.nt * 128, kvrow,
+                      pol_last);
+        }
+        ++items;
+        const int nm = it.m_hi - it.m_lo + 1;
+        for (int st = 0; st < it.n && ok; ++st) {
+          const int h = it.kvh * p.group + st / nm;
+          const int m = it.m_lo + st % nm;
+          const uint32_t slot = lidx % C::NST;
+          if (!wait_bounded(BAR(B_QEMPTY + slot), ((lidx / C::NST) & 1) ^ 1, abort_flag, tmo)) { ok = false; break; }
+          const uint32_t stage = sbase + C::OFF_RING + slot * 2 * C::TILE_BYTES;
+          const int bh = it.b * p.H + h;
+          mbar_expect_tx(BAR(B_QFULL + slot), 2 * C::TILE_BYTES + 1024);
+          for (int pn = 0; pn < C::NPANEL; ++pn) {
+            tma_load_3d(stage + pn * C::PANEL_BYTES, &tm_q, BAR(B_QFULL + slot), pn * 64, m * 128, bh, pol_last);
+            tma_load_3d(stage + C::TILE_BYTES + pn * C::PANEL_BYTES, &tm_do, BAR(B_QFULL + slot), pn * 64, m * 128,
+                        bh, pol_last);
+          }
+          // LSE and Dv of the 128 rows (padded arrays: 512-byte aligned rows)
+          const size_t roff = static_cast<size_t>(bh) * p.Sq_pad + static_cast<size_t>(m) * 128;
+          const uint32_t rows_dst = sbase + C::OFF_ROWS + slot * 1024;
+          bulk_load(rows_dst, p.lse2 + roff, 512, BAR(B_QFULL + slot));
+          bulk_load(rows_dst + 512, p.dvec + roff, 512, BAR(B_QFULL + slot));
+          ++lidx;
+        }
+      }
+      // drain this thread's copies
+      if (items > 0) drain_bounded(BAR(B_KVFULL), (items - 1) & 1, tmo);
+      for (uint32_t idx = (lidx > C::NST ? lidx - C::NST : 0); idx < lidx; ++idx)
+        drain_bounded(BAR(B_QFULL + idx % C::NST), (idx / C::NST) & 1, tmo);
+    }
+  } else if (warp == kBwdMmaWarp) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t tS = tbase + C::T_S, tDP = tbase + C::T_DP, tDV = tbase + C::T_ACC0, tDK = tbase + C::T_ACC1;
+      const uint64_t dk_k = make_sdesc_sw128(sbase + C::OFF_A, 16, 1024);       // K as K-major A
+      const uint64_t dv_k = make_sdesc_sw128(sbase + C::OFF_B, 16, 1024);       // V as K-major A
+      const uint64_t dring_k = make_sdesc_sw128(sbase + C::OFF_RING, 16, 1024);           // K-major B
+      const uint64_t dring_mn = make_sdesc_sw128(sbase + C::OFF_RING, C::PANEL_BYTES, 1024);  // MN-major B
+      auto ss = [&](uint32_t dst, uint64_t a0, uint64_t b0) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int col = kk * 16;
+          const uint32_t off = ((col / 64) * C::PANEL_BYTES + (col % 64) * 2) >> 4;
+          mma_f16_ss(dst, a0 + off, b0 + off, C::IDESC_SS, kk > 0);
+        }
+      };
+      auto ts = [&](uint32_t dst, uint32_t a_tmem, uint64_t b0, bool acc) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_f16_ts(dst, a_tmem + kk * 8, b0 + ((kk * 16 * 128) >> 4), C::IDESC_TS, (acc || kk > 0) ? 1u : 0u);
+      };
+      uint32_t items = 0, cidx = 0, tcount = 0;
+      bool ok = true;
+      for (int r = 0; ok; ++r) {
+        const int w = sched_pos(r, cta, G);
+        if (w >= p.num_items) break;
+        const KvItem it = make_kv_item(p, w);
+        if (it.n == 0) continue;
+        if (!wait_bounded(BAR(B_KVFULL), items & 1, abort_flag, tmo)) { ok = false; break; }
+        tc_fence_after();
+        for (int st = 0; st < it.n; ++st) {
+          const uint32_t slot = (cidx + st) % C::NST;
+          const uint32_t t = tcount + st;
+          if (!wait_bounded(BAR(B_QFULL + slot), ((cidx + st) / C::NST) & 1, abort_flag, tmo)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t soff = (slot * 2 * C::TILE_BYTES) >> 4;
+          // S^T = K Q^T and dP^T = V dO^T (they overwrite P^T / dS^T of the previous step,
+          // which that step's dV / dK MMAs, issued earlier by this thread, read first)
+          ss(tS, dk_k, dring_k + soff);
+          ss(tDP, dv_k, dring_k + soff + (C::TILE_BYTES >> 4));
+          mma_commit(BAR(B_SFULL));
+          if (!wait_bounded(BAR(B_PFULL), t & 1, abort_flag, tmo)) { ok = false; break; }
+          tc_fence_after();
+          // dV += P^T dO,  dK += dS^T Q
+          ts(tDV, tS, dring_mn + soff + (C::TILE_BYTES >> 4), st > 0);
+          ts(tDK, tDP, dring_mn + soff, st > 0);
+          mma_commit(BAR(B_QEMPTY + slot));
+        }
+        if (!ok) break;
+        mma_commit(BAR(B_KVEMPTY));
+        mma_commit(BAR(B_DONE));
+        cidx += it.n;
+        tcount += it.n;
+        ++items;
+      }
+      mma_commit(BAR(B_DRAIN));
+      drain_bounded(BAR(B_DRAIN), 0, tmo);
+    }
+  } else {
+    // ------------------------------------------------------------------ compute warps
+    const int rloc = warp * 32 + lane;                       // key row within the tile (TMEM lane)
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t tS = tbase + C::T_S + lane_off, tDP = tbase + C::T_DP + lane_off;
+    const uint32_t tDV = tbase + C::T_ACC0 + lane_off, tDK = tbase + C::T_ACC1 + lane_off;
+    const float* srows = reinterpret_cast<const float*>(sptr + C::OFF_ROWS);
+    uint32_t tcount = 0, cidx = 0, items = 0;
+    bool ok = true;
+    for (int r = 0; ok; ++r) {
+      const int w = sched_pos(r, cta, G);
+      if (w >= p.num_items) break;
+      const KvItem it = make_kv_item(p, w);
+      const int j = it.nt * 128 + rloc;                      // key position
+      if (it.n == 0) {
+        // no query row sees this key tile: dK = dV = 0
+        if (j < p.Sk) {
+          const size_t orow = (static_cast<size_t>(it.b * p.Hkv + it.kvh) * p.Sk + j) * D;
+          for (int c = 0; c < D; c += 8) {
+            *reinterpret_cast<uint4*>(p.dv + orow + c) = make_uint4(0u, 0u, 0u, 0u);
+            *reinterpret_cast<uint4*>(p.dk + orow + c) = make_uint4(0u, 0u, 0u, 0u);
+          }
+        }
+        continue;
+      }
+      const int2 rs = rows_seeing_key(p, j);
+      int ilo = rs.x, ihi = min(rs.y, p.Sq - 1);
+      if (j >= p.Sk) ihi = -1;                               // padding key: sees nothing
+      const bool has_doc = p.doc != nullptr;
+      bool doc_elem = false;
+      int doc_j = 0;
+      const int* drow = has_doc ? p.doc + static_cast<size_t>(it.b) * p.Sk : nullptr;
+      if (has_doc && j < p.Sk) {
+        if (p.doc_sorted != nullptr && __ldg(p.doc_sorted + it.b)) {
+          const int2 run = doc_run(drow, p.Sk, j);
+          ilo = max(ilo, run.x);
+          ihi = min(ihi, run.y);
+        } else {
+          doc_elem = true;
+          doc_j = __ldg(drow + j);
+        }
+      }
+      const int nm = it.m_hi - it.m_lo + 1;
+      const int d = p.Sk - p.Sq;
+      for (int st = 0; st < it.n; ++st) {
+        const int h = it.kvh * p.group + st / nm;
+        const int m = it.m_lo + st % nm;
+        const uint32_t slot = (cidx + st) % C::NST;
+        const uint32_t t = tcount + st;
+        float slope_l2 = 0.f;
+        if constexpr (ALIBI) slope_l2 = __ldg(p.alibi + h) * kLog2e;
+        // the stage's rows of LSE and Dv came by bulk copy: observe that copy's barrier too
+        if (!__all_sync(0xffffffffu, wait_bounded(BAR(B_QFULL + slot), ((cidx + st) / C::NST) & 1, abort_flag, tmo) &&
+                                     wait_bounded(BAR(B_SFULL), t & 1, abort_flag, tmo))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const float* lse2 = srows + slot * 256;
+        const float* dvv = lse2 + 128;
+        // visible query columns of this key row within tile m
+        uint32_t vm[4];
+        interval_mask(ilo - m * 128, ihi - m * 128, vm);
+        const float rel0 = static_cast<float>(j - d - m * 128);    // j - i' for column 0
+        uint32_t pf[64];                                           // bf16 pairs of P * dt/ds
+        // pass 1: P^T = exp2(t - lse2) over S^T's first 64 columns
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t sv[32];
+          tmem_ld_x32_wait(tS + 32 * c, sv);
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const int col = 32 * c + e;
+            float f0, f1;
+            float t0 = bwd_modify<SOFTCAP, ALIBI>(p, __uint_as_float(sv[e]), slope_l2, rel0 - col, &f0);
+            float t1 = bwd_modify<SOFTCAP, ALIBI>(p, __uint_as_float(sv[e + 1]), slope_l2, rel0 - col - 1, &f1);
+            bool v0 = ((vm[col >> 5] >> (col & 31)) & 1u) != 0u;
+            bool v1 = ((vm[(col + 1) >> 5] >> ((col + 1) & 31)) & 1u) != 0u;
+            if (doc_elem) {
+              const int i0 = m * 128 + col;
+              v0 = v0 && i0 < p.Sq && __ldg(drow + min(i0, p.Sq - 1)) == doc_j;
+              v1 = v1 && i0 + 1 < p.Sq && __ldg(drow + min(i0 + 1, p.Sq - 1)) == doc_j;
+            }
+            const float p0 = v0 ? ex2_approx(t0 - lse2[col]) : 0.f;
+            const float p1 = v1 ? ex2_approx(t1 - lse2[col + 1]) : 0.f;
+            pk[e >> 1] = pack_bf16x2(p0, p1);
+            pf[(32 * c + e) >> 1] = pack_bf16x2(p0 * f0, p1 * f1);
+          }
+          tmem_st_x16_nowait<0>(tS + 16 * c, pk);
+        }
+        // pass 2: dS^T = (P dt/ds) (dP^T - Dv) over dP^T's first 64 columns
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t dv[32];
+          tmem_ld_x32_wait(tDP + 32 * c, dv);
+          uint32_t dk[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const int col = 32 * c + e;
+            const float2 pp = unpack_bf16x2(pf[col >> 1]);
+            const float ds0 = pp.x * (__uint_as_float(dv[e]) - dvv[col]);
+            const float ds1 = pp.y * (__uint_as_float(dv[e + 1]) - dvv[col + 1]);
+            dk[e >> 1] = pack_bf16x2(ds0, ds1);
+          }
+          tmem_st_x16_nowait<0>(tDP + 16 * c, dk);
+        }
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        tc_fence_before();
+        mbar_arrive(BAR(B_PFULL));
+      }
+      if (!__all_sync(0xffffffffu, ok && !*abort_flag)) {
+        ok = false;
+        break;
+      }
+      // ---- epilogue: dV and scale * dK -> bf16
+      if (!__all_sync(0xffffffffu, wait_bounded(BAR(B_DONE), items & 1, abort_flag, tmo))) { ok = false; break; }
+      tc_fence_after();
+      const size_t orow = (static_cast<size_t>(it.b * p.Hkv + it.kvh) * p.Sk + j) * D;
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        __nv_bfloat16* dst = (which == 0 ? p.dv : p.dk) + orow;
+        const float mul = which == 0 ? 1.f : p.scale;
+        const uint32_t src = which == 0 ? tDV : tDK;
+#pragma unroll
+        for (int ch = 0; ch < D / 32; ++ch) {
+          uint32_t a[32];
+          tmem_ld_x32_wait(src + ch * 32, a);
+          uint32_t wv[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c)
+            wv[c] = pack_bf16x2(__uint_as_float(a[2 * c]) * mul, __uint_as_float(a[2 * c + 1]) * mul);
+          if (j < p.Sk) {
+            uint4* o4 = reinterpret_cast<uint4*>(dst + ch * 32);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) o4[v] = make_uint4(wv[4 * v], wv[4 * v + 1], wv[4 * v + 2], wv[4 * v + 3]);
+          }
+        }
+      }
+      tc_fence_before();
+      cidx += it.n;
+      tcount += it.n;
+      ++items;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kBwdMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tbase, C::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// dQ kernel
+// ---------------------------------------------------------------------------------------
+struct QItem {
+  int b, h, bh, mt;    // batch, head, b*H+h, query tile
+  int kt_lo, n;        // key tiles kt_lo .. kt_lo + n - 1
+};
+
+__device__ __forceinline__ QItem make_q_item(const BwdParams& p, int w) {
+  QItem it;
+  const int BH = p.B * p.H;
+  if (p.lpt) {   // causal: the last query tiles see the most key tiles
+    it.mt = p.nqt - 1 - w / BH;
+    it.bh = w % BH;
+  } else {
+    it.bh = w / p.nqt;
+    it.mt = w % p.nqt;
+  }
+  it.b = it.bh / p.H;
+  it.h = it.bh % p.H;
+  const int i0 = it.mt * 128, i1 = min(i0 + 127, p.Sq - 1);
+  int c0 = max(keys_seen_by_row(p, i0).x, 0);
+  int c1 = min(keys_seen_by_row(p, i1).y, p.Sk - 1);
+  if (p.mask_kind & 1) c0 = max(c0, 0);
+  if (p.doc != nullptr && p.doc_sorted != nullptr && __ldg(p.doc_sorted + it.b)) {
+    const int* drow = p.doc + static_cast<size_t>(it.b) * p.Sk;
+    c0 = max(c0, doc_run(drow, p.Sk, i0).x);
+    c1 = min(c1, doc_run(drow, p.Sk, i1).y);
+  }
+  if (c1 < c0) {
+    it.kt_lo = 0;
+    it.n = 0;
+    return it;
+  }
+  it.kt_lo = c0 / 128;
+  it.n = c1 / 128 - it.kt_lo + 1;
+  return it;
+}
+
+template <int D, bool SOFTCAP, bool ALIBI>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                   const BwdParams p) {
+  using C = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* sptr = smem_raw + (sbase - raw);
+  auto BAR = [&](int i) -> uint32_t { return sbase + C::OFF_BAR + 8 * i; };
+  constexpr int B_QFULL = 0, B_QEMPTY = 1, B_KVFULL = 2, B_KVEMPTY = 2 + C::NST, B_SFULL = 2 + 2 * C::NST,
+                B_PFULL = B_SFULL + 1, B_DONE = B_PFULL + 1, B_DRAIN = B_DONE + 1;
+  static_assert(B_DRAIN < C::NBAR, "barrier count");
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sptr + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sptr + C::OFF_MISC + 4);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = gridDim.x, cta = blockIdx.x;
+  const unsigned long long tmo = p.timeout_ns;
+
+  if (threadIdx.x == 0) {
+    mbar_init(BAR(B_QFULL), 1);
+    mbar_init(BAR(B_QEMPTY), 1);
+    for (int s = 0; s < C::NST; ++s) {
+      mbar_init(BAR(B_KVFULL + s), 1);
+      mbar_init(BAR(B_KVEMPTY + s), 1);
+    }
+    mbar_init(BAR(B_SFULL), 1);
+    mbar_init(BAR(B_PFULL), 128);
+    mbar_init(BAR(B_DONE), 1);
+    mbar_init(BAR(B_DRAIN), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kBwdMmaWarp) {
+    tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == kBwdLoadWarp && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_do);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_holder;
+
+  if (warp == kBwdLoadWarp) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const uint64_t pol_last = policy_evict_last();
+      const uint64_t pol_first = policy_evict_first();
+      uint32_t items = 0, lidx = 0;
+      bool ok = true;
+      for (int r = 0; ok; ++r) {
+        const int w = sched_pos(r, cta, G);
+        if (w >= p.num_items) break;
+        const QItem it = make_q_item(p, w);
+        if (it.n == 0) continue;
+        if (items > 0 && !wait_bounded(BAR(B_QEMPTY), (items - 1) & 1, abort_flag, tmo)) break;
+        mbar_expect_tx(BAR(B_QFULL), 2 * C::TILE_BYTES);
+        for (int pn = 0; pn < C::NPANEL; ++pn) {
+          tma_load_3d(sbase + C::OFF_A + pn * C::PANEL_BYTES, &tm_q, BAR(B_QFULL), pn * 64, it.mt * 128, it.bh,
+                      pol_first);
+          tma_load_3d(sbase + C::OFF_B + pn * C::PANEL_BYTES, &tm_do, BAR(B_QFULL), pn * 64, it.mt * 128, it.bh,
+                      pol_first);
+        }
+        ++items;
+        const int kvrow = it.b * p.Hkv + it.h / p.group;
+        for (int st = 0; st < it.n && ok; ++st) {
+          const int kt = it.kt_lo + st;
+          const uint32_t slot = lidx % C::NST;
+          if (!wait_bounded(BAR(B_KVEMPTY + slot), ((lidx / C::NST) & 1) ^ 1, abort_flag, tmo)) { ok = false; break; }
+          const uint32_t stage = sbase + C::OFF_RING + slot * 2 * C::TILE_BYTES;
+          mbar_expect_tx(BAR(B_KVFULL + slot), 2 * C::TILE_BYTES);
+          for (int pn = 0; pn < C::NPANEL; ++pn) {
+            tma_load_3d(stage + pn * C::PANEL_BYTES, &tm_k, BAR(B_KVFULL + slot), pn * 64, kt * 128, kvrow, pol_last);
+            tma_load_3d(stage + C::TILE_BYTES + pn * C::PANEL_BYTES, &tm_v, BAR(B_KVFULL + slot), pn * 64, kt * 128,
+                        kvrow, pol_last);
+          }
+          ++lidx;
+        }
+      }
+      if (items > 0) drain_bounded(BAR(B_QFULL), (items - 1) & 1, tmo);
+      for (uint32_t idx = (lidx > C::NST ? lidx - C::NST : 0); idx < lidx; ++idx)
+        drain_bounded(BAR(B_KVFULL + idx % C::NST), (idx / C::NST) & 1, tmo);
+    }
+  } else if (warp == kBwdMmaWarp) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t tS = tbase + C::T_S, tDP = tbase + C::T_DP, tDQ = tbase + C::T_ACC0;
+      const uint64_t dq_k = make_sdesc_sw128(sbase + C::OFF_A, 16, 1024);
+      const uint64_t ddo_k = make_sdesc_sw128(sbase + C::OFF_B, 16, 1024);
+      const uint64_t dring_k = make_sdesc_sw128(sbase + C::OFF_RING, 16, 1024);
+      const uint64_t dring_mn = make_sdesc_sw128(sbase + C::OFF_RING, C::PANEL_BYTES, 1024);
+      auto ss = [&](uint32_t dst, uint64_t a0, uint64_t b0) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int col = kk * 16;
+          const uint32_t off = ((col / 64) * C::PANEL_BYTES + (col % 64) * 2) >> 4;
+          mma_f16_ss(dst, a0 + off, b0 + off, C::IDESC_SS, kk > 0);
+        }
+      };
+      uint32_t items = 0, cidx = 0, tcount = 0;
+      bool ok = true;
+      for (int r = 0; ok; ++r) {
+        const int w = sched_pos(r, cta, G);
+        if (w >= p.num_items) break;
+        const QItem it = make_q_item(p, w);
+        if (it.n == 0) continue;
+        if (!wait_bounded(BAR(B_QFULL), items & 1, abort_flag, tmo)) { ok = false; break; }
+        tc_fence_after();
+        for (int st = 0; st < it.n; ++st) {
+          const uint32_t slot = (cidx + st) % C::NST;
+          const uint32_t t = tcount + st;
+          if (!wait_bounded(BAR(B_KVFULL + slot), ((cidx + st) / C::NST) & 1, abort_flag, tmo)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t soff = (slot * 2 * C::TILE_BYTES) >> 4;
+          ss(tS, dq_k, dring_k + soff);                                  // S = Q K^T
+          ss(tDP, ddo_k, dring_k + soff + (C::TILE_BYTES >> 4));         // dP = dO V^T
+          mma_commit(BAR(B_SFULL));
+          if (!wait_bounded(BAR(B_PFULL), t & 1, abort_flag, tmo)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)                                 // dQ += dS K
+            mma_f16_ts(tDQ, tDP + kk * 8, dring_mn + soff + ((kk * 16 * 128) >> 4), C::IDESC_TS,
+                       (st > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(BAR(B_KVEMPTY + slot));
+        }
+        if (!ok) break;
+        mma_commit(BAR(B_QEMPTY));
+        mma_commit(BAR(B_DONE));
+        cidx += it.n;
+        tcount += it.n;
+        ++items;
+      }
+      mma_commit(BAR(B_DRAIN));
+      drain_bounded(BAR(B_DRAIN), 0, tmo);
+    }
+  } else {
+    // ------------------------------------------------------------------ compute warps
+    const int rloc = warp * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t tS = tbase + C::T_S + lane_off, tDP = tbase + C::T_DP + lane_off;
+    const uint32_t tDQ = tbase + C::T_ACC0 + lane_off;
+    uint32_t tcount = 0, items = 0;
+    bool ok = true;
+    for (int r = 0; ok; ++r) {
+      const int w = sched_pos(r, cta, G);
+      if (w >= p.num_items) break;
+      const QItem it = make_q_item(p, w);
+      const int i = it.mt * 128 + rloc;
+      if (it.n == 0) {
+        // rows that see no key: dQ = 0
+        if (i < p.Sq) {
+          __nv_bfloat16* dst = p.dq + (static_cast<size_t>(it.bh) * p.Sq + i) * D;
+          for (int c = 0; c < D; c += 8) *reinterpret_cast<uint4*>(dst + c) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        continue;
+      }
+      const int2 ks = keys_seen_by_row(p, i);
+      int jlo = ks.x, jhi = min(ks.y, p.Sk - 1);
+      if (i >= p.Sq) jhi = -1;
+      const bool has_doc = p.doc != nullptr;
+      bool doc_elem = false;
+      int doc_i = 0;
+      const int* drow = has_doc ? p.doc + static_cast<size_t>(it.b) * p.Sk : nullptr;
+      if (has_doc && i < p.Sq) {
+        if (p.doc_sorted != nullptr && __ldg(p.doc_sorted + it.b)) {
+          const int2 run = doc_run(drow, p.Sk, i);
+          jlo = max(jlo, run.x);
+          jhi = min(jhi, run.y);
+        } else {
+          doc_elem = true;
+          doc_i = __ldg(drow + i);
+        }
+      }
+      const size_t rr = static_cast<size_t>(it.bh) * p.Sq_pad + i;
+      const float lse2 = __ldg(p.lse2 + rr);
+      const float dvi = __ldg(p.dvec + rr);
+      float slope_l2 = 0.f;
+      if constexpr (ALIBI) slope_l2 = __ldg(p.alibi + it.h) * kLog2e;
+      const int ip = i + p.Sk - p.Sq;
+      for (int st = 0; st < it.n; ++st) {
+        const uint32_t t = tcount + st;
+        const int kt = it.kt_lo + st;
+        if (!__all_sync(0xffffffffu, wait_bounded(BAR(B_SFULL), t & 1, abort_flag, tmo))) { ok = false; break; }
+        tc_fence_after();
+        uint32_t vm[4];
+        interval_mask(jlo - kt * 128, jhi - kt * 128, vm);
+        const float rel0 = static_cast<float>(kt * 128 - ip);      // j - i' for column 0
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t sv[32], dv[32];
+          tmem_ld_x32_wait(tS + 32 * c, sv);
+          tmem_ld_x32_wait(tDP + 32 * c, dv);
+          uint32_t dk[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const int col = 32 * c + e;
+            float f0, f1;
+            const float t0 = bwd_modify<SOFTCAP, ALIBI>(p, __uint_as_float(sv[e]), slope_l2, rel0 + col, &f0);
+            const float t1 = bwd_modify<SOFTCAP, ALIBI>(p, __uint_as_float(sv[e + 1]), slope_l2, rel0 + col + 1, &f1);
+            bool v0 = ((vm[col >> 5] >> (col & 31)) & 1u) != 0u;
+            bool v1 = ((vm[(col + 1) >> 5] >> ((col + 1) & 31)) & 1u) != 0u;
+            if (doc_elem) {
+              const int j0 = kt * 128 + col;
+              v0 = v0 && j0 < p.Sk && __ldg(drow + min(j0, p.Sk - 1)) == doc_i;
+              v1 = v1 && j0 + 1 < p.Sk && __ldg(drow + min(j0 + 1, p.Sk - 1)) == doc_i;
+            }
+            const float p0 = v0 ? ex2_approx(t0 - lse2) : 0.f;
+            const float p1 = v1 ? ex2_approx(t1 - lse2) : 0.f;
+            // P * dt/ds rounded to bf16 first, as in the dK/dV kernel, so that both kernels
+            // use the same dS
+            const float2 pp = unpack_bf16x2(pack_bf16x2(p0 * f0, p1 * f1));
+            dk[e >> 1] = pack_bf16x2(pp.x * (__uint_as_float(dv[e]) - dvi), pp.y * (__uint_as_float(dv[e + 1]) - dvi));
+          }
+          tmem_st_x16_nowait<0>(tDP + 16 * c, dk);
+        }
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        tc_fence_before();
+        mbar_arrive(BAR(B_PFULL));
+      }
+      if (!__all_sync(0xffffffffu, ok && !*abort_flag)) {
+        ok = false;
+        break;
+      }
+      if (!__all_sync(0xffffffffu, wait_bounded(BAR(B_DONE), items & 1, abort_flag, tmo))) { ok = false; break; }
+      tc_fence_after();
+      __nv_bfloat16* dst = p.dq + (static_cast<size_t>(it.bh) * p.Sq + i) * D;
+#pragma unroll
+      for (int ch = 0; ch < D / 32; ++ch) {
+        uint32_t a[32];
+        tmem_ld_x32_wait(tDQ + ch * 32, a);
+        uint32_t wv[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+          wv[c] = pack_bf16x2(__uint_as_float(a[2 * c]) * p.scale, __uint_as_float(a[2 * c + 1]) * p.scale);
+        if (i < p.Sq) {
+          uint4* o4 = reinterpret_cast<uint4*>(dst + ch * 32);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) o4[v] = make_uint4(wv[4 * v], wv[4 * v + 1], wv[4 * v + 2], wv[4 * v + 3]);
+        }
+      }
+      tc_fence_before();
+      tcount += it.n;
+      ++items;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kBwdMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tbase, C::TMEM_COLS);
+  }
+}
+
+}  // namespace attn
