@@ -442,6 +442,42 @@ def per_config_record(ta, name, dev, peaks, min_ms=60.0, min_launches=10):
     return rec
 
 
+def bwd_record(ta, name, dev, peaks, min_ms=60.0):
+    """The backward of a workload (dQ, dK, dV from the forward's O and LSE and a random
+    dO): device time of one attn_bwd call (its three launches) and TFLOP/s over the
+    algorithmic 10 * D FLOPs per visible pair (five matrix products: Q K^T, dO V^T, P^T dO,
+    dS^T Q, dS K; the kernels recompute two of them to avoid atomics, 14 * D done)."""
+    w = WORKLOADS[name]
+    case = Case(ta, w, dev, seed=0)
+    case.step()
+    g = torch.Generator().manual_seed(1)
+    do = torch.randn(case.o.shape, generator=g).to(torch.bfloat16).to(dev)
+    dq, dk, dv = (torch.empty_like(t) for t in (case.q, case.k, case.v))
+
+    def bstep():
+        ta.attn_bwd(case.q, case.k, case.v, case.o, case.lse, do, dq, dk, dv, scale=w.scale, mask_kind=w.mask_kind,
+                    window=w.window, softcap=w.softcap, alibi_slopes=case.sl, doc_ids=case.doc, stream=case.stream)
+
+    for _ in range(3):
+        bstep()
+    torch.cuda.synchronize(dev)
+    t1 = time_launches(bstep, 2, case.stream, dev)
+    n = max(10, int(min_ms / max(min(t1), 1e-3)))
+    ms = time_launches(bstep, n, case.stream, dev)
+    if ta.attn_get_status(case.stream) != 0:
+        raise SystemExit(f"kernel status error in the backward of {name}")
+    mean_ms = float(np.mean(ms))
+    flops = 2.5 * algorithmic_flops(w)
+    tflops = flops / (mean_ms * 1e-3) / 1e12
+    rec = {"workload": w.note + ", backward", "launches": n, "ms": mean_ms, "tflops_exact": tflops,
+           "peak_tflops": peaks["bf16"], "frac": tflops / peaks["bf16"],
+           "flops": "10*D per visible pair (14*D executed: S and dP are recomputed for dQ)",
+           "launches_per_call": 3}
+    del case, do, dq, dk, dv
+    torch.cuda.empty_cache()
+    return rec
+
+
 def sustained_record(case, dev, peaks, local, seconds=1.5):
     """Back-to-back launches for about ``seconds`` (long enough for the power cap to act),
     with its own NVML clock record, against the sustained peak."""
@@ -649,6 +685,7 @@ def main():
             del case
             torch.cuda.empty_cache()
             line["per_config"] = {name: per_config_record(ta, name, dev, peaks) for name in WORKLOADS}
+            line["per_config"]["causal_backward"] = bwd_record(ta, "causal", dev, peaks)
         if world == 1 and not args.no_cpu_baseline:
             f, dt, desc = oracle_sample(w, args.cpu_budget)
             line["cpu_baseline"] = {"value": f / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
