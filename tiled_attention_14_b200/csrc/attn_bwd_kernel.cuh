@@ -74,7 +74,10 @@ struct BwdCfg {
   static constexpr int OFF_BAR = OFF_ROWS + NST * 1024;
   static constexpr int NBAR = 16;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  // At least 120 KB so that two CTAs never share an SM: each allocates all 512 TMEM
+  // columns, and a second CTA on the SM would wait for the first one's to be freed.
+  static constexpr int SMEM_USED = OFF_MISC + 16 + 1024;
+  static constexpr int SMEM_BYTES = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t T_S = 0, T_DP = 128, T_ACC0 = 256, T_ACC1 = 256 + D;
   static constexpr uint32_t IDESC_SS = make_idesc(1u, 128, 128, false);   // 128x128, both K-major
