@@ -546,6 +546,9 @@ def main():
                     help="time the device steps only (no e2e, sustained, per-config or CPU legs): "
                          "the command the ncu captures run")
     ap.add_argument("--heads", type=int, default=0, help="override H (smaller ncu captures)")
+    ap.add_argument("--tau", type=float, default=None,
+                    help="ablation builds only (TILED_ATTENTION_LIB=.../libattn_abl*.so): rescale threshold; "
+                         "the line then reports the rescale counters")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -572,8 +575,16 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
 
     import tiled_attention_14_b200 as ta
-    ta._lib.load()
+    lib = ta._lib.load()
     dev = torch.device("cuda", local)
+    ablation = None
+    if args.tau is not None:
+        import ctypes
+        lib.attn_ablation_set.restype, lib.attn_ablation_set.argtypes = ctypes.c_int, [ctypes.c_float]
+        lib.attn_ablation_counts.restype, lib.attn_ablation_counts.argtypes = ctypes.c_int, [ctypes.c_void_p]
+        lib.attn_ablation_sw_exp_every.restype = ctypes.c_int
+        ablation = {"tau": args.tau, "sw_exp_every": lib.attn_ablation_sw_exp_every(),
+                    "lib": os.path.basename(os.environ.get("TILED_ATTENTION_LIB", ""))}
     case = Case(ta, w, dev, seed=rank)
     stream = case.stream
     quant_ms = case.quantize_ms() if w.fp8 else None
@@ -583,6 +594,9 @@ def main():
     torch.cuda.synchronize(dev)
     if ta.attn_get_status(stream) != 0:
         raise SystemExit("kernel status error during warm-up")
+    if ablation is not None:
+        if lib.attn_ablation_set(args.tau) != 0:
+            raise SystemExit("attn_ablation_set failed")
 
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -609,12 +623,22 @@ def main():
     flops = algorithmic_flops(w)
     total_ms = max_over_ranks(total_ms, dist, dev)
     value = weak_scaling_value(flops, args.steps, world, total_ms)
+    if ablation is not None:
+        import ctypes
+        cnt = (ctypes.c_ulonglong * 2)()
+        if lib.attn_ablation_counts(ctypes.addressof(cnt)) != 0:
+            raise SystemExit("attn_ablation_counts failed")
+        ablation.update(rescale_steps_per_launch=cnt[0] / args.steps, row_steps_per_launch=cnt[1] / args.steps,
+                        rescale_fraction=cnt[0] / max(cnt[1], 1))
     if args.kernel_only:
         if rank == 0:
-            print(json.dumps({"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
-                              "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
-                              "config": workload_config(w), "kernel_only": True,
-                              "gpu_launches": case.launches_per_step * args.steps}), flush=True)
+            line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+                    "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+                    "config": workload_config(w), "kernel_only": True,
+                    "gpu_launches": case.launches_per_step * args.steps}
+            if ablation is not None:
+                line["ablation"] = ablation
+            print(json.dumps(line), flush=True)
         if dist:
             dist.barrier()
             dist.destroy_process_group()

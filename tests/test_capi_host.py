@@ -94,3 +94,33 @@ def test_binding_rejects_host_tensors_and_bad_outputs():
         ta.attn_fwd(meta, meta, meta)
     with pytest.raises(ValueError):
         ta.attn_quantize_e4m3(torch.zeros(1, 1, 128, 128))
+
+
+ABL_SIGNATURES = {
+    "attn_ablation_set": (ctypes.c_int, [ctypes.c_float]),
+    "attn_ablation_counts": (ctypes.c_int, [ctypes.c_void_p]),
+    "attn_ablation_sw_exp_every": (ctypes.c_int, []),
+}
+
+
+def test_ablation_builds_export_their_header():
+    """The ablation builds export attn.h's symbols and include/attn_ablation.h's; the product
+    build exports none of the latter."""
+    from tiled_attention_14_b200 import build
+    src = open(os.path.join(ROOT, "include", "attn_ablation.h")).read()
+    names = set(re.findall(r"ATTN_API\s+[\w\s\*]+?\b(attn_\w+)\s*\(", src))
+    assert names == set(ABL_SIGNATURES)
+    for so in build.ABLATIONS:
+        lib = _lib.open_library(os.path.join(os.path.dirname(_lib.LIB_PATH), so))
+        for n in names:
+            assert getattr(lib, n) is not None
+        fn = lib.attn_ablation_sw_exp_every
+        fn.restype = ctypes.c_int
+        assert fn() == (4 if "sw4" in so else 0)
+        set_tau = lib.attn_ablation_set
+        set_tau.restype, set_tau.argtypes = ABL_SIGNATURES["attn_ablation_set"]
+        assert set_tau(9.0) == _lib.ATTN_ERR_INVALID and set_tau(-1.0) == _lib.ATTN_ERR_INVALID
+    product = _lib.load()
+    for n in names:
+        with pytest.raises(AttributeError):
+            getattr(product, n)

@@ -50,20 +50,27 @@ class AttnError(RuntimeError):
         super().__init__(f"{what}: {strerror(code)} ({code})")
 
 
-def load() -> ctypes.CDLL:
-    """Loads the in-tree libattn.so (raises if it is missing: there is no fallback)."""
-    global _lib
-    if _lib is not None:
-        return _lib
-    if not os.path.exists(LIB_PATH):
-        raise RuntimeError(f"{LIB_PATH} is missing; build it with `python -m tiled_attention_14_b200.build`")
-    lib = ctypes.CDLL(LIB_PATH)
+def open_library(path: str) -> ctypes.CDLL:
+    """Opens a build of libattn.so at ``path`` with the ctypes signatures of include/attn.h."""
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing; build it with `python -m tiled_attention_14_b200.build`")
+    lib = ctypes.CDLL(path)
     for name, (res, args) in SIGNATURES.items():
         fn = getattr(lib, name)
         fn.restype = res
         fn.argtypes = args
-    _lib = lib
     return lib
+
+
+def load() -> ctypes.CDLL:
+    """Loads the in-tree libattn.so (raises if it is missing: there is no fallback).  The
+    environment variable TILED_ATTENTION_LIB may name another build of the same sources
+    (the ablation builds) for measurements."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    _lib = open_library(os.environ.get("TILED_ATTENTION_LIB") or LIB_PATH)
+    return _lib
 
 
 def strerror(code: int) -> str:

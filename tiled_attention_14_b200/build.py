@@ -29,21 +29,38 @@ def _nvcc() -> str:
 
 def _deps() -> list[str]:
     files = [os.path.join(CSRC, f) for f in os.listdir(CSRC)]
-    files.append(os.path.join(INCLUDE, "attn.h"))
+    files += [os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE)]
     return files
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+# Ablation builds (test and measurement only, never the product path): the same sources with
+# ATTN_ABLATION (runtime rescale threshold, rescale counters, include/attn_ablation.h) and
+# optionally the software exp2 on one element pair in four.
+ABLATIONS = {
+    "libattn_abl.so": ["-DATTN_ABLATION"],
+    "libattn_abl_sw4.so": ["-DATTN_ABLATION", "-DATTN_SW_EXP_EVERY=4"],
+}
+
+
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(f) <= t for f in _deps())
 
 
-def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> str:
-    if not force and up_to_date():
-        return LIB
-    tmp = LIB + ".tmp"
+def build_ablations(force: bool = False, verbose: bool = False) -> list[str]:
+    out = []
+    for name, flags in ABLATIONS.items():
+        out.append(build(force=force, verbose=verbose, extra=flags, lib=os.path.join(HERE, name)))
+    return out
+
+
+def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None, lib: str = LIB) -> str:
+    if not force and up_to_date(lib):
+        return lib
+    LIB_OUT = lib
+    tmp = LIB_OUT + ".tmp"
     cmd = [_nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
            "-shared", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
            "-I", INCLUDE, "-I", CSRC, "--expt-relaxed-constexpr",
@@ -58,8 +75,8 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
     check_registers(res.stderr)
     if verbose:
         sys.stderr.write(res.stderr)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, LIB_OUT)
+    return LIB_OUT
 
 
 # Registers per thread the attention kernels must be compiled to: the kernel's setmaxnreg
@@ -89,3 +106,5 @@ def check_registers(ptxas_log: str) -> None:
 
 if __name__ == "__main__":
     build(force="--force" in sys.argv, verbose="--ptxas-v" in sys.argv)
+    if "--ablations" in sys.argv:
+        build_ablations(force="--force" in sys.argv)

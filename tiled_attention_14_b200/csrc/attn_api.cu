@@ -13,6 +13,9 @@
 #include <mutex>
 
 #include "attn.h"
+#ifdef ATTN_ABLATION
+#include "attn_ablation.h"
+#endif
 #include "attn_bwd_kernel.cuh"
 #include "attn_fwd_kernel.cuh"
 #include "quant_kernel.cuh"
@@ -172,9 +175,27 @@ FwdParams make_params(void* o, float* lse, int B, int H, int Hkv, int Sq, int Sk
   p.num_items = static_cast<int>(items);
   // Causal without a window: query blocks differ a lot in length -> longest first.
   p.lpt_qb_major = ((mask_kind & ATTN_MASK_CAUSAL) && !(mask_kind & (ATTN_MASK_WINDOW | ATTN_MASK_DOC))) ? 1 : 0;
+  p.lpt_heads = 0;
   p.fault_skip = g_fault_skip.load();
   p.timeout_ns = static_cast<unsigned long long>(g_timeout_ms.load()) * 1000000ull;
   return p;
+}
+
+#ifndef ATTN_L2_GROUP_BYTES
+#define ATTN_L2_GROUP_BYTES (32ll << 20)
+#endif
+// Causal longest-first order works through groups of heads whose K and V together take at
+// most ATTN_L2_GROUP_BYTES (a quarter of the 126 MB L2), so the K/V tiles that the CTAs in
+// flight re-read come from L2 rather than HBM.  Heads that share K/V (grouped-query) count
+// once per key/value head.  0 turns grouping off.
+int lpt_head_group(const FwdParams& p, int Sk, int D, int eb) {
+  if (!p.lpt_qb_major || ATTN_L2_GROUP_BYTES <= 0) return 0;
+  const long long kv_head = 2ll * Sk * D * eb;
+  long long kv_heads = ATTN_L2_GROUP_BYTES / (kv_head > 0 ? kv_head : 1);
+  if (kv_heads < 1) kv_heads = 1;
+  long long heads = kv_heads * p.group;          // query heads per group
+  const long long BH = static_cast<long long>(p.B) * p.H;
+  return heads >= BH ? 0 : static_cast<int>(heads);
 }
 
 int launch_tile_map(int* counts, uint32_t* entries, int B, int Sq, int Sk, int mask_kind, int window,
@@ -222,6 +243,7 @@ int run_fwd(bool fp8, const void* q, const void* k, const void* v, const float* 
     p.nsb_q = (Sq + 127) / 128;
     p.nsb_k = (Sk + 127) / 128;
   }
+  p.lpt_heads = lpt_head_group(p, Sk, D, fp8 ? 1 : 2);
   CUtensorMap tq, tk, tv;
   if (encode_map(&tq, q, fp8, B * H, Sq, D) != ATTN_OK || encode_map(&tk, k, fp8, B * Hkv, Sk, D) != ATTN_OK ||
       encode_map(&tv, v, fp8, B * Hkv, Sk, D) != ATTN_OK)
@@ -300,6 +322,7 @@ int run_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float*
   if (need_map && (rc = noalloc_scratch(dev, &scratch)) != ATTN_OK) return rc;
 
   FwdParams p = make_params(o, lse, B, H, H, Sq, Sk, scale, mask_kind, window, softcap, alibi, doc_ids);
+  p.lpt_heads = lpt_head_group(p, Sk, D, 2);
   CUtensorMap tq, tk, tv;
   if (encode_map(&tq, q, false, B * H, Sq, D) != ATTN_OK || encode_map(&tk, k, false, B * H, Sk, D) != ATTN_OK ||
       encode_map(&tv, v, false, B * H, Sk, D) != ATTN_OK)
@@ -343,6 +366,7 @@ int run_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* 
   p.cu_k = cu_k;
   p.Tq = total_q;
   p.Tk = total_k;
+  p.lpt_heads = lpt_head_group(p, max_sk, D, 2);
   CUtensorMap tq, tk, tv;
   if (encode_map_thd(&tq, q, H, total_q, D) != ATTN_OK || encode_map_thd(&tk, k, Hkv, total_k, D) != ATTN_OK ||
       encode_map_thd(&tv, v, Hkv, total_k, D) != ATTN_OK)
@@ -599,6 +623,30 @@ void attn_shutdown(void) {
   cudaMemPool_t pool;
   if (cudaDeviceGetDefaultMemPool(&pool, dev) == cudaSuccess) cudaMemPoolTrimTo(pool, 0);
 }
+
+#ifdef ATTN_ABLATION
+int attn_ablation_set(float tau) {
+  if (!std::isfinite(tau) || tau < 0.f || tau > 8.f) return ATTN_ERR_INVALID;   // P <= 2^tau <= 256
+  int dev = 0;
+  const int rc = current_device(&dev);
+  if (rc != ATTN_OK) return rc;
+  const unsigned long long zero[2] = {0ull, 0ull};
+  if (cudaMemcpyToSymbol(attn::g_abl_tau, &tau, sizeof(float)) != cudaSuccess ||
+      cudaMemcpyToSymbol(attn::g_abl_counts, zero, sizeof(zero)) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  return ATTN_OK;
+}
+
+int attn_ablation_counts(unsigned long long* out) {
+  if (!out) return ATTN_ERR_INVALID;
+  if (cudaDeviceSynchronize() != cudaSuccess) return ATTN_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(out, attn::g_abl_counts, 2 * sizeof(unsigned long long)) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  return ATTN_OK;
+}
+
+int attn_ablation_sw_exp_every(void) { return attn::kSwExpEvery; }
+#endif
 
 void attn_debug_set_fault(int skip_signal, int timeout_ms) {
   g_fault_skip.store(skip_signal ? 1 : 0);

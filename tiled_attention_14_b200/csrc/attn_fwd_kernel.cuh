@@ -62,8 +62,12 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kNegInf = -__builtin_huge_valf();
 
 // Software exp2 (FMA pipes) takes one element pair in kSwExpEvery (0: all on MUFU).  Measured on
-// B200: with the packed-f32x2 softmax the exponentials are not MUFU-bound, so it is off.
-constexpr int kSwExpEvery = 0;
+// B200: with the packed-f32x2 softmax the exponentials are not MUFU-bound, so the product build
+// has it off; the ablation build (ATTN_ABLATION) compiles it in with ATTN_SW_EXP_EVERY.
+#ifndef ATTN_SW_EXP_EVERY
+#define ATTN_SW_EXP_EVERY 0
+#endif
+constexpr int kSwExpEvery = ATTN_SW_EXP_EVERY;
 constexpr int kSwDiv = kSwExpEvery > 0 ? kSwExpEvery : 1;
 // Coefficients of 2^f on [-1/2, 1/2] (near-minimax in relative error, fitted by
 // tiled_attention_14_b200/fit_exp2_poly.py; max relative error 7.5e-5 in float32).
@@ -74,6 +78,21 @@ constexpr float kE3 = 0.0551716685295105f;
 
 // Device status word (one per device that loads the library).
 __device__ int g_attn_status;
+
+#ifdef ATTN_ABLATION
+// Ablation build only: the rescale threshold comes from device memory, and every (row, key
+// tile) step of the softmax is counted — [0] steps that rescaled, [1] steps of rows that had
+// seen a visible key.
+__device__ float g_abl_tau = 8.0f;
+__device__ unsigned long long g_abl_counts[2];
+#endif
+__device__ __forceinline__ float rescale_tau() {
+#ifdef ATTN_ABLATION
+  return *reinterpret_cast<volatile float*>(&g_abl_tau);
+#else
+  return kTau;
+#endif
+}
 
 struct FwdParams {
   __nv_bfloat16* o;
@@ -101,6 +120,7 @@ struct FwdParams {
   int nsb_q, nsb_k;
   int num_items;           // B * H * nqb work items
   int lpt_qb_major;        // 1: order work by query block first (causal: longest first)
+  int lpt_heads;           // ... within groups of this many (b, h) heads (0: one group)
   int fault_skip;          // test hook: group 1 skips its first P-ready signal
   unsigned long long timeout_ns;
 };
@@ -243,8 +263,15 @@ __device__ __forceinline__ Item make_item(const FwdParams& p, int w) {
   Item it;
   const int BH = p.B * p.H;   // packed sequences: B is the number of sequences
   if (p.lpt_qb_major) {
-    it.qb = p.nqb - 1 - w / BH;
-    it.bh = w % BH;
+    // Longest first within groups of lpt_heads heads, so that the K/V of the heads in
+    // flight stay in L2; groups follow one another (the last one may be smaller).
+    const int HG = p.lpt_heads > 0 ? p.lpt_heads : BH;
+    const int g = w / (HG * p.nqb);
+    const int base = g * HG;
+    const int hg = min(HG, BH - base);
+    const int r = w - base * p.nqb;
+    it.qb = p.nqb - 1 - r / hg;
+    it.bh = base + r % hg;
   } else {
     it.bh = w / p.nqb;
     it.qb = p.nqb - 1 - w % p.nqb;
@@ -436,7 +463,7 @@ __device__ __forceinline__ void softmax_tile(const FwdParams& p, const Item& it,
       // ---- online softmax with the rescale threshold
       bool rescale = false;
       float alpha = 1.f;
-      if (mx > m_run + kTau) {
+      if (mx > m_run + rescale_tau()) {
         if (m_run != kNegInf) {
           alpha = ex2_approx(m_run - mx);
           rescale = true;
@@ -444,6 +471,15 @@ __device__ __forceinline__ void softmax_tile(const FwdParams& p, const Item& it,
         }
         m_run = mx;
       }
+#ifdef ATTN_ABLATION
+      {
+        const unsigned r = __ballot_sync(0xffffffffu, rescale), v = __ballot_sync(0xffffffffu, m_run != kNegInf);
+        if ((threadIdx.x & 31) == 0) {
+          atomicAdd(&g_abl_counts[0], static_cast<unsigned long long>(__popc(r)));
+          atomicAdd(&g_abl_counts[1], static_cast<unsigned long long>(__popc(v)));
+        }
+      }
+#endif
       const float msub = (m_run == kNegInf) ? 0.f : m_run;
       // ---- exponentials, packed two per register (f32x2 FMA / ADD), P to TMEM in two halves
       const float2 sc2 = make_float2(sc, sc);
