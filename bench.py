@@ -334,27 +334,26 @@ class Case:
         self.launches_per_step = 2 if w.doc else 1
         if w.fp8:
             # e4m3 operands with per-128-row scales, quantised once (the quantiser is timed alone)
-            self.q8 = [ta.attn_quantize_e4m3(t, stream=self.stream) for t in (self.q, self.k, self.v)]
+            self.q8 = [ta.attn_quantize_e4m3(t) for t in (self.q, self.k, self.v)]
 
     def run(self, q, k, v, quantize=False):
         """The public call a user makes for this workload, on the given inputs."""
         w, ta = self.w, self.ta
         if w.fp8:
             if quantize:
-                a8 = [ta.attn_quantize_e4m3(t, stream=self.stream) for t in (q, k, v)]
+                a8 = [ta.attn_quantize_e4m3(t) for t in (q, k, v)]
             else:
                 a8 = self.q8
             (q8, qs), (k8, ks), (v8, vs) = a8
             ta.attn_fwd_fp8(q8, k8, v8, qs, ks, vs, o=self.o, lse=self.lse, scale=w.scale,
-                            mask_kind=w.mask_kind, stream=self.stream)
+                            mask_kind=w.mask_kind)
         elif w.varlen:
             ta.attn_fwd_varlen(q, k, v, self.cu, self.cu, self.maxlen, self.maxlen, o=self.o, lse=self.lse,
                                scale=w.scale, mask_kind=w.mask_kind, window=w.window, softcap=w.softcap,
-                               alibi_slopes=self.sl, stream=self.stream)
+                               alibi_slopes=self.sl)
         else:
             ta.attn_fwd(q, k, v, o=self.o, lse=self.lse, scale=w.scale, mask_kind=w.mask_kind,
-                        window=w.window, softcap=w.softcap, alibi_slopes=self.sl, doc_ids=self.doc,
-                        stream=self.stream)
+                        window=w.window, softcap=w.softcap, alibi_slopes=self.sl, doc_ids=self.doc)
 
     def step(self):
         self.run(self.q, self.k, self.v)
@@ -383,8 +382,9 @@ class Case:
 
 
 def time_launches(step, n, stream, dev, flush=None):
-    """Per-launch device times (ms) of n steps, each bracketed by events on the launching
-    stream; with ``flush`` (a buffer larger than L2) L2 is overwritten before every step."""
+    """Per-launch device times (ms) of n eager steps, each bracketed by events on the
+    launching stream; with ``flush`` (a buffer larger than L2) L2 is overwritten before every
+    step.  Host work between the events counts, so this is for long steps only."""
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
     for i in range(n):
@@ -395,6 +395,61 @@ def time_launches(step, n, stream, dev, flush=None):
         ends[i].record(stream)
     torch.cuda.synchronize(dev)
     return [s.elapsed_time(e) for s, e in zip(starts, ends)]
+
+
+def capture(fn, n, dev):
+    """A CUDA graph of n calls of fn (the calls run on torch's capture stream, which the
+    library takes as the current stream), or None if capture is not possible."""
+    try:
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(side):
+            fn()
+        torch.cuda.current_stream(dev).wait_stream(side)
+        torch.cuda.synchronize(dev)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(n):
+                fn()
+        torch.cuda.synchronize(dev)
+        return g
+    except Exception as e:  # pragma: no cover - reported in the line as eager timing
+        print(f"graph capture failed ({e}); timing eager launches", file=sys.stderr)
+        torch.cuda.synchronize(dev)
+        return None
+
+
+def time_steps(step, n, dev, flush=None):
+    """Device time (ms) of n steps replayed from one CUDA graph, bracketed by events: no host
+    work between the launches.  With ``flush`` every step is preceded by an L2 flush inside
+    the graph, and a graph of the flushes alone is timed and subtracted.  Returns
+    (ms per step, "graph" | "eager")."""
+    stream = torch.cuda.current_stream(dev)
+    body = step if flush is None else (lambda: (flush.add_(1), step()))
+    g = capture(body, n, dev)
+    if g is None:
+        ms = time_launches(step, n, stream, dev, flush)
+        return float(np.mean(ms)), "eager"
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g.replay()                     # first replay uploads the graph
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    total = e0.elapsed_time(e1)
+    if flush is not None:
+        gf = capture(lambda: flush.add_(1), n, dev)
+        gf.replay()
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        gf.replay()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        total -= e0.elapsed_time(e1)
+        del gf
+    del g
+    return total / n, "graph"
 
 
 def compulsory_bytes(w) -> int:
@@ -413,20 +468,19 @@ def per_config_record(ta, name, dev, peaks, min_ms=60.0, min_launches=10):
     for _ in range(3):
         case.step()
     torch.cuda.synchronize(dev)
-    t1 = time_launches(case.step, 2, case.stream, dev)
-    n = max(min_launches, int(min_ms / max(min(t1), 1e-3)))
+    t1, _ = time_steps(case.step, 2, dev)
+    n = max(min_launches, int(min_ms / max(t1, 1e-3)))
     flush = None
     if compulsory_bytes(w) < L2_BYTES:
         flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
-    ms = time_launches(case.step, n, case.stream, dev, flush)
-    if ta.attn_get_status(case.stream) != 0:
+    mean_ms, how = time_steps(case.step, n, dev, flush)
+    if ta.attn_get_status() != 0:
         raise SystemExit(f"kernel status error in workload {name}")
-    mean_ms = float(np.mean(ms))
     flops = algorithmic_flops(w)
     tflops = flops / (mean_ms * 1e-3) / 1e12
     peak = peaks["fp8"] if w.fp8 else peaks["bf16"]
     gbs = compulsory_bytes(w) / (mean_ms * 1e-3) / 1e9
-    rec = {"workload": w.note, "launches": n, "ms": mean_ms, "ms_min": float(np.min(ms)),
+    rec = {"workload": w.note, "steps": n, "timing": how, "ms": mean_ms,
            "tflops_exact": tflops, "peak_tflops": peak, "frac": tflops / peak,
            "dtype": "e4m3" if w.fp8 else "bf16", "compulsory_bytes": compulsory_bytes(w),
            "gbs_compulsory": gbs, "hbm_frac": gbs / peaks["hbm"],
@@ -456,20 +510,19 @@ def bwd_record(ta, name, dev, peaks, min_ms=60.0):
 
     def bstep():
         ta.attn_bwd(case.q, case.k, case.v, case.o, case.lse, do, dq, dk, dv, scale=w.scale, mask_kind=w.mask_kind,
-                    window=w.window, softcap=w.softcap, alibi_slopes=case.sl, doc_ids=case.doc, stream=case.stream)
+                    window=w.window, softcap=w.softcap, alibi_slopes=case.sl, doc_ids=case.doc)
 
     for _ in range(3):
         bstep()
     torch.cuda.synchronize(dev)
-    t1 = time_launches(bstep, 2, case.stream, dev)
-    n = max(10, int(min_ms / max(min(t1), 1e-3)))
-    ms = time_launches(bstep, n, case.stream, dev)
-    if ta.attn_get_status(case.stream) != 0:
+    t1, _ = time_steps(bstep, 2, dev)
+    n = max(10, int(min_ms / max(t1, 1e-3)))
+    mean_ms, how = time_steps(bstep, n, dev)
+    if ta.attn_get_status() != 0:
         raise SystemExit(f"kernel status error in the backward of {name}")
-    mean_ms = float(np.mean(ms))
     flops = 2.5 * algorithmic_flops(w)
     tflops = flops / (mean_ms * 1e-3) / 1e12
-    rec = {"workload": w.note + ", backward", "launches": n, "ms": mean_ms, "tflops_exact": tflops,
+    rec = {"workload": w.note + ", backward", "steps": n, "timing": how, "ms": mean_ms, "tflops_exact": tflops,
            "peak_tflops": peaks["bf16"], "frac": tflops / peaks["bf16"],
            "flops": "10*D per visible pair (14*D executed: S and dP are recomputed for dQ)",
            "launches_per_call": 3}
@@ -481,16 +534,25 @@ def bwd_record(ta, name, dev, peaks, min_ms=60.0):
 def sustained_record(case, dev, peaks, local, seconds=1.5):
     """Back-to-back launches for about ``seconds`` (long enough for the power cap to act),
     with its own NVML clock record, against the sustained peak."""
-    t = time_launches(case.step, 3, case.stream, dev)
-    n = max(20, int(seconds * 1e3 / max(float(np.mean(t)), 1e-3)))
+    t, _ = time_steps(case.step, 3, dev)
+    per_graph = max(10, int(100.0 / max(t, 1e-3)))            # about 100 ms per replay
+    reps = max(2, int(seconds * 1e3 / (per_graph * max(t, 1e-3))))
+    g = capture(case.step, per_graph, dev)
+    stream = torch.cuda.current_stream(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local, period_s=0.02) as clocks:
-        e0.record(case.stream)
-        for _ in range(n):
-            case.step()
-        e1.record(case.stream)
+        e0.record(stream)
+        for _ in range(reps):
+            if g is not None:
+                g.replay()
+            else:
+                for _ in range(per_graph):
+                    case.step()
+        e1.record(stream)
         torch.cuda.synchronize(dev)
     ms = e0.elapsed_time(e1)
+    n = reps * per_graph
+    del g
     tflops = algorithmic_flops(case.w) * n / (ms * 1e-3) / 1e12
     peak = peaks["fp8_sustained"] if case.w.fp8 else peaks["bf16_sustained"]
     return {"launches": n, "ms_total": ms, "tflops_exact": tflops, "peak_tflops": peak,
@@ -586,7 +648,7 @@ def main():
         ablation = {"tau": args.tau, "sw_exp_every": lib.attn_ablation_sw_exp_every(),
                     "lib": os.path.basename(os.environ.get("TILED_ATTENTION_LIB", ""))}
     case = Case(ta, w, dev, seed=rank)
-    stream = case.stream
+    stream = torch.cuda.current_stream(dev)
     quant_ms = case.quantize_ms() if w.fp8 else None
 
     for _ in range(args.warmup):
@@ -598,8 +660,9 @@ def main():
         if lib.attn_ablation_set(args.tau) != 0:
             raise SystemExit("attn_ablation_set failed")
 
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    # The K timed steps are one CUDA graph (captured after the warm-up, not timed), so the
+    # device runs them back to back with no host work between launches.
+    graph = capture(case.step, args.steps, dev)
     if dist:
         dist.barrier()
     torch.cuda.synchronize(dev)
@@ -607,16 +670,18 @@ def main():
     t_end = torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clocks:
         t_begin.record(stream)
-        for i in range(args.steps):
-            starts[i].record(stream)
-            case.step()
-            ends[i].record(stream)
+        if graph is not None:
+            graph.replay()
+        else:
+            for _ in range(args.steps):
+                case.step()
         t_end.record(stream)
         torch.cuda.synchronize(dev)
     if dist:
         dist.barrier()
     total_ms = t_begin.elapsed_time(t_end)
-    per_launch_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    timing = "cuda graph of the K steps" if graph is not None else "eager launches"
+    del graph
     if ta.attn_get_status(stream) != 0:
         raise SystemExit("kernel status error in the timed region")
 
@@ -680,7 +745,7 @@ def main():
     if rank == 0:
         peaks = measured_peaks()
         # the attention kernel is the dominant launch (one launch per step for analytic masks)
-        launch_ms = float(np.mean(per_launch_ms))
+        launch_ms = total_ms / args.steps
         achieved = flops / (launch_ms * 1e-3) / 1e12
         peak = peaks["fp8"] if w.fp8 else peaks["bf16"]
         line = {
@@ -700,6 +765,7 @@ def main():
                     "d2h_bytes_per_step": d2h},
             "clocks": clocks.summary(),
             "gpu_launches": case.launches_per_step * args.steps,
+            "timing": timing,
         }
         if quant_ms is not None:
             line["quantize_ms_per_tensor_set"] = quant_ms

@@ -58,7 +58,8 @@ typedef enum {
   ATTN_ERR_UNSUPPORTED = -2,  /* device is not sm_100 */
   ATTN_ERR_CUDA = -3,         /* a CUDA runtime/driver call or launch failed */
   ATTN_ERR_TIMEOUT = -4,      /* a kernel's bounded wait ran out (from attn_get_status) */
-  ATTN_ERR_NOMEM = -5         /* workspace allocation failed */
+  ATTN_ERR_NOMEM = -5,        /* workspace allocation failed */
+  ATTN_ERR_CHECK = -6         /* debug build only: a TMA or TMEM bounds check failed in a kernel */
 } attn_status;
 
 enum {

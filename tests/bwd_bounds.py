@@ -16,8 +16,8 @@ forward output's own rounding on Dv (O is bf16: |dDv_i| <= 2^-8 sum_d |dO_id O_i
     dK_j :  T = scale * sum_i (|dS_ij| + P_ij f'_ij A_i) |Q_i|,   A_i = sum_d |dO_id O_id|
     dQ_i :  T = scale * sum_j (|dS_ij| + P_ij f'_ij A_i) |K_j|
 
-eps = 2^-7 covers two bf16 roundings (2^-9 each) with margin and the LSE error of the
-forward (about 1e-6 in natural-log units).  A wrong or dropped term moves g by about |g|
+eps = 2^-7 + 2^-10 covers two bf16 roundings of a term (half an ulp, 2^-8 each: bf16 keeps
+8 significant bits) and the LSE error of the forward (about 1e-6 in natural-log units).  A wrong or dropped term moves g by about |g|
 itself, far outside the bound.
 """
 from __future__ import annotations
@@ -27,7 +27,7 @@ import numpy as np
 from oracle.attention import _f64, modified_scores, softmax_rows, visible_mask
 from oracle.attention_bwd import attention_bwd
 
-EPS = 2.0 ** -7
+EPS = 2.0 ** -7 + 2.0 ** -10
 REL_OUT = 2.0 ** -8
 ATOL = 1e-5
 

@@ -16,7 +16,7 @@ import torch
 
 from attn_workloads import MASK_CAUSAL, MASK_NONE, alibi_slopes, make_qkv
 from oracle.attention import modified_scores, visible_mask
-from tests.gpu_helpers import compare, oracle, to_dev
+from tests.gpu_helpers import compare, oracle_eav, to_dev
 from tiled_attention_14_b200 import _lib
 from tiled_attention_14_b200.build import ABLATIONS
 
@@ -66,8 +66,8 @@ def test_ablation_builds_match_the_oracle(name, tau):
         qd, kd, vd, sld = to_dev(q, k, v, sl)
         o, lse = _fwd(lib, qd, kd, vd, c["mask"], c.get("softcap", 0.0), sld)
         torch.cuda.synchronize()
-        O, L = oracle(q, k, v, 1.0 / math.sqrt(128), c["mask"], 0, c.get("softcap", 0.0), sl)
-        compare(o, lse, O, L, tol_rel=2.0 ** -8 if c["q_mul"] > 1 else 0.0)
+        O, L, E = oracle_eav(q, k, v, 1.0 / math.sqrt(128), c["mask"], 0, c.get("softcap", 0.0), sl)
+        compare(o, lse, O, L, eav=E)
 
 
 def _expected_counts(q, k, scale, mask, tau):

@@ -11,7 +11,7 @@ import torch
 
 from attn_workloads import (MASK_CAUSAL, MASK_DOC, MASK_NONE, MASK_WINDOW, WORKLOADS, alibi_slopes,
                             doc_ids_from_lengths, make_doc_ids, make_qkv, sample_rows)
-from tests.gpu_helpers import TOL_REL_STRESS, compare, oracle, to_dev
+from tests.gpu_helpers import compare, oracle_eav, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -27,8 +27,8 @@ def _run(B, H, Sq, Sk, D, mask=MASK_NONE, window=0, softcap=0.0, alibi=False, do
                          alibi_slopes=sld, doc_ids=docd)
     torch.cuda.synchronize()
     assert ta.attn_get_status() == 0
-    O, L = oracle(q, k, v, scale, mask, window, softcap, sl, doc)
-    return compare(o, lse, O, L, tol_rel=TOL_REL_STRESS if q_mul > 1.0 else 0.0)
+    O, L, E = oracle_eav(q, k, v, scale, mask, window, softcap, sl, doc)
+    return compare(o, lse, O, L, eav=E)
 
 
 def test_tiny_config():
@@ -117,8 +117,8 @@ def _sampled(w, n_random=24, q_mul=1.0):
                          softcap=w.softcap, alibi_slopes=sld, doc_ids=docd)
     torch.cuda.synchronize()
     assert ta.attn_get_status() == 0
-    O, L = oracle(q, k, v, w.scale, w.mask_kind, w.window, w.softcap, sl, doc, rows=rows)
-    return compare(o, lse, O, L, rows=rows)
+    O, L, E = oracle_eav(q, k, v, w.scale, w.mask_kind, w.window, w.softcap, sl, doc, rows=rows)
+    return compare(o, lse, O, L, rows=rows, eav=E)
 
 
 @pytest.mark.parametrize("name", ["causal", "window", "alibi", "softcap", "doc", "long"])

@@ -8,7 +8,7 @@ import pytest
 import torch
 
 from attn_workloads import MASK_CAUSAL, make_qkv
-from tests.gpu_helpers import compare, oracle, to_dev
+from tests.gpu_helpers import compare, oracle_eav, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -31,5 +31,5 @@ def test_skipped_signal_times_out_and_context_survives():
     o, lse = ta.attn_fwd(qd, kd, vd, mask_kind=MASK_CAUSAL)
     torch.cuda.synchronize()
     assert ta.attn_get_status() == _lib.ATTN_OK
-    O, L = oracle(q, k, v, 1.0 / 128 ** 0.5, MASK_CAUSAL)
-    compare(o, lse, O, L)
+    O, L, E = oracle_eav(q, k, v, 1.0 / 128 ** 0.5, MASK_CAUSAL)
+    compare(o, lse, O, L, eav=E)

@@ -46,7 +46,8 @@ def _pool_high_water(reset: bool) -> int:
     assert err == rt.cudaError_t.cudaSuccess
     attr = rt.cudaMemPoolAttr.cudaMemPoolAttrUsedMemHigh
     if reset:
-        (err,) = rt.cudaMemPoolSetAttribute(pool, attr, rt.cuuint64_t(0))
+        from cuda.bindings import driver as drv
+        (err,) = rt.cudaMemPoolSetAttribute(pool, attr, drv.cuuint64_t(0))
         assert err == rt.cudaError_t.cudaSuccess
     err, val = rt.cudaMemPoolGetAttribute(pool, attr)
     assert err == rt.cudaError_t.cudaSuccess

@@ -14,6 +14,7 @@ ATTN_ERR_UNSUPPORTED = -2
 ATTN_ERR_CUDA = -3
 ATTN_ERR_TIMEOUT = -4
 ATTN_ERR_NOMEM = -5
+ATTN_ERR_CHECK = -6
 
 MASK_NONE = 0
 MASK_CAUSAL = 1

@@ -49,9 +49,15 @@ def up_to_date(lib: str = LIB) -> bool:
     return all(os.path.getmtime(f) <= t for f in _deps())
 
 
+# Debug build (tests only): every TMA copy and TMEM move bounds-checked in the kernels, a failed
+# check recorded as ATTN_ERR_CHECK in the status word instead of a fault.
+DEBUG = {"libattn_debug.so": ["-DATTN_DEBUG_CHECKS"]}
+
+
 def build_ablations(force: bool = False, verbose: bool = False) -> list[str]:
+    """Builds the ablation libraries and the bounds-checked debug library."""
     out = []
-    for name, flags in ABLATIONS.items():
+    for name, flags in {**ABLATIONS, **DEBUG}.items():
         out.append(build(force=force, verbose=verbose, extra=flags, lib=os.path.join(HERE, name)))
     return out
 

@@ -613,6 +613,7 @@ const char* attn_strerror(int code) {
     case ATTN_ERR_CUDA: return "CUDA error";
     case ATTN_ERR_TIMEOUT: return "a bounded wait inside a kernel ran out";
     case ATTN_ERR_NOMEM: return "workspace allocation failed";
+    case ATTN_ERR_CHECK: return "a bounds check of the debug build failed inside a kernel";
     default: return "unknown status";
   }
 }

@@ -76,8 +76,6 @@ constexpr float kE1 = 0.6932609677314758f;
 constexpr float kE2 = 0.2426111400127411f;
 constexpr float kE3 = 0.0551716685295105f;
 
-// Device status word (one per device that loads the library).
-__device__ int g_attn_status;
 
 #ifdef ATTN_ABLATION
 // Ablation build only: the rescale threshold comes from device memory, and every (row, key
@@ -240,7 +238,8 @@ __device__ __forceinline__ bool drain_bounded(uint32_t bar, uint32_t parity,
 // ---------------------------------------------------------------------------------------
 struct Item {
   int b, h, bh, qb;
-  int kvbh;       // key/value head row of the K/V tensors (b * Hkv + h / group)
+  int kvh;        // key/value head (h / group)
+  int kvbh;       // key/value head row of batched K/V tensors (b * Hkv + kvh)
   int sq, sk;     // query and key lengths of this item's sequence
   int q_off, k_off;  // first query / key token of the sequence (packed layout; else 0)
   int n;          // number of key tiles visited
@@ -278,7 +277,8 @@ __device__ __forceinline__ Item make_item(const FwdParams& p, int w) {
   }
   it.b = it.bh / p.H;
   it.h = it.bh % p.H;
-  it.kvbh = it.b * p.Hkv + it.h / p.group;
+  it.kvh = it.h / p.group;
+  it.kvbh = it.b * p.Hkv + it.kvh;
   if (p.cu_q != nullptr) {
     it.q_off = __ldg(p.cu_q + it.b);
     it.sq = __ldg(p.cu_q + it.b + 1) - it.q_off;
@@ -642,7 +642,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             mbar_expect_tx(BAR(B_KVFULL + slot), C::TILE_BYTES);
             const CUtensorMap* tm = kv ? &tm_v : &tm_k;
-            const int kc1 = varlen ? it.kvbh : kt * 128, kc2 = varlen ? it.k_off + kt * 128 : it.kvbh;
+            const int kc1 = varlen ? it.kvh : kt * 128, kc2 = varlen ? it.k_off + kt * 128 : it.kvbh;
             for (int pn = 0; pn < C::NPANEL; ++pn)
               tma_load_3d(sbase + C::OFF_KV + slot * C::TILE_BYTES + pn * C::PANEL_BYTES, tm,
                           BAR(B_KVFULL + slot), pn * C::PANEL_COLS, kc1, kc2, pol_kv);

@@ -7,12 +7,53 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
-#include "tmem_moves.cuh"
-
 namespace attn {
+
+// Device status word (one per device that loads the library): 0, or the first error code a
+// kernel recorded (ATTN_ERR_* of attn.h).
+__device__ int g_attn_status;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ---------------------------------------------------------------------------------------
+// Debug build (ATTN_DEBUG_CHECKS): every TMA copy and TMEM move is checked before it is
+// issued — shared-memory destination inside the CTA's dynamic allocation and aligned, tensor
+// coordinates non-negative with the innermost one on a 16-byte boundary, TMEM column range
+// inside the 512 columns and the lane quarter the warp may access.  A failed check records
+// ATTN_ERR_CHECK in the status word and skips the access (loads then leave their barrier
+// short, so the bounded waits end the kernel); nothing traps.  The product build compiles
+// the checks away.
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ bool debug_check(bool ok) {
+#ifdef ATTN_DEBUG_CHECKS
+  if (!ok) atomicCAS(&g_attn_status, 0, -6 /* ATTN_ERR_CHECK */);
+  return ok;
+#else
+  (void)ok;
+  return true;
+#endif
+}
+__device__ __forceinline__ uint32_t dynamic_smem_bytes() {
+  uint32_t n;
+  asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(n));
+  return n;
+}
+__device__ __forceinline__ uint32_t dynamic_smem_base() {
+  extern __shared__ uint8_t attn_dyn_smem[];
+  return smem_u32(attn_dyn_smem);
+}
+// shared-memory range [dst, dst + bytes) inside the dynamic allocation, dst aligned to `align`
+__device__ __forceinline__ bool smem_range_ok(uint32_t dst, uint32_t bytes, uint32_t align) {
+  const uint32_t base = dynamic_smem_base();
+  return (dst & (align - 1)) == 0 && dst >= base && dst + bytes <= base + dynamic_smem_bytes();
+}
+// TMEM move of `cols` 32-bit columns from `taddr` by this warp (32x32b shape)
+__device__ __forceinline__ bool tmem_range_ok(uint32_t taddr, uint32_t cols) {
+  const uint32_t col = taddr & 0xFFFFu, lane = taddr >> 16;
+  const uint32_t warp_q = (threadIdx.x >> 5) & 3u;
+  return col + cols <= 512u && lane == 32u * warp_q;
 }
 
 __device__ __forceinline__ uint64_t global_timer_ns() {
@@ -20,6 +61,12 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
+
+}  // namespace attn
+
+#include "tmem_moves.cuh"
+
+namespace attn {
 
 // ---------------------------------------------------------------------------------------
 // mbarrier
@@ -58,6 +105,11 @@ __device__ __forceinline__ void tma_prefetch_desc(const void* map) {
 }
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* map, uint32_t bar, int c0,
                                             int c1, int c2, uint64_t policy) {
+#ifdef ATTN_DEBUG_CHECKS
+  // boxes are 128 rows of 128 bytes, 128-byte swizzled (1024-byte aligned destination)
+  if (!debug_check(smem_range_ok(dst, 128u * 128u, 1024u) && c0 >= 0 && (c0 % 16) == 0 && c1 >= 0 && c2 >= 0))
+    return;
+#endif
   asm volatile(
       "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
       " [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(dst),
@@ -67,6 +119,11 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* map, uint3
 // Untiled bulk copy global -> shared (both addresses 16-byte aligned, bytes a multiple of 16),
 // completing `bytes` of transaction count on the mbarrier; no multicast.
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+#ifdef ATTN_DEBUG_CHECKS
+  if (!debug_check(smem_range_ok(dst, bytes, 16u) && (reinterpret_cast<uintptr_t>(src) & 15u) == 0 &&
+                   (bytes & 15u) == 0))
+    return;
+#endif
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
       "l"(src), "r"(bytes), "r"(bar)

@@ -10,6 +10,12 @@ namespace attn {
 // store (or tcgen05.wait::st) before the data is handed to the tensor core, and the
 // stored registers are not rewritten before that.
 __device__ __forceinline__ void tmem_ld_x16_wait(uint32_t taddr, uint32_t (&r)[16]) {
+#ifdef ATTN_DEBUG_CHECKS
+  if (!debug_check(tmem_range_ok(taddr, 16))) {
+    for (int i = 0; i < 16; ++i) r[i] = 0u;
+    return;
+  }
+#endif
   asm volatile(
     "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];\n\t"
     "tcgen05.wait::ld.sync.aligned;\n"
@@ -17,6 +23,12 @@ __device__ __forceinline__ void tmem_ld_x16_wait(uint32_t taddr, uint32_t (&r)[1
     : "r"(taddr) : "memory");
 }
 __device__ __forceinline__ void tmem_ld_x32_wait(uint32_t taddr, uint32_t (&r)[32]) {
+#ifdef ATTN_DEBUG_CHECKS
+  if (!debug_check(tmem_range_ok(taddr, 32))) {
+    for (int i = 0; i < 32; ++i) r[i] = 0u;
+    return;
+  }
+#endif
   asm volatile(
     "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
     "tcgen05.wait::ld.sync.aligned;\n"
@@ -24,6 +36,12 @@ __device__ __forceinline__ void tmem_ld_x32_wait(uint32_t taddr, uint32_t (&r)[3
     : "r"(taddr) : "memory");
 }
 __device__ __forceinline__ void tmem_ld_x64_wait(uint32_t taddr, uint32_t (&r)[64]) {
+#ifdef ATTN_DEBUG_CHECKS
+  if (!debug_check(tmem_range_ok(taddr, 64))) {
+    for (int i = 0; i < 64; ++i) r[i] = 0u;
+    return;
+  }
+#endif
   asm volatile(
     "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];\n\t"
     "tcgen05.wait::ld.sync.aligned;\n"
@@ -31,6 +49,12 @@ __device__ __forceinline__ void tmem_ld_x64_wait(uint32_t taddr, uint32_t (&r)[6
     : "r"(taddr) : "memory");
 }
 __device__ __forceinline__ void tmem_ld_x128_wait(uint32_t taddr, uint32_t (&r)[128]) {
+#ifdef ATTN_DEBUG_CHECKS
+  if (!debug_check(tmem_range_ok(taddr, 128))) {
+    for (int i = 0; i < 128; ++i) r[i] = 0u;
+    return;
+  }
+#endif
   asm volatile(
     "tcgen05.ld.sync.aligned.32x32b.x128.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63, %64, %65, %66, %67, %68, %69, %70, %71, %72, %73, %74, %75, %76, %77, %78, %79, %80, %81, %82, %83, %84, %85, %86, %87, %88, %89, %90, %91, %92, %93, %94, %95, %96, %97, %98, %99, %100, %101, %102, %103, %104, %105, %106, %107, %108, %109, %110, %111, %112, %113, %114, %115, %116, %117, %118, %119, %120, %121, %122, %123, %124, %125, %126, %127}, [%128];\n\t"
     "tcgen05.wait::ld.sync.aligned;\n"
@@ -40,6 +64,11 @@ __device__ __forceinline__ void tmem_ld_x128_wait(uint32_t taddr, uint32_t (&r)[
 template <int OFF, int N>
 __device__ __forceinline__ void tmem_st_x16_nowait(uint32_t taddr, const uint32_t (&r)[N]) {
   static_assert(OFF + 16 <= N, "slice out of range");
+#ifdef ATTN_DEBUG_CHECKS
+  if (!debug_check(tmem_range_ok(taddr, 16))) {
+    return;
+  }
+#endif
   asm volatile(
     "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};\n\t"
     :: "r"(taddr), "r"(r[OFF + 0]), "r"(r[OFF + 1]), "r"(r[OFF + 2]), "r"(r[OFF + 3]), "r"(r[OFF + 4]), "r"(r[OFF + 5]), "r"(r[OFF + 6]), "r"(r[OFF + 7]), "r"(r[OFF + 8]), "r"(r[OFF + 9]), "r"(r[OFF + 10]), "r"(r[OFF + 11]), "r"(r[OFF + 12]), "r"(r[OFF + 13]), "r"(r[OFF + 14]), "r"(r[OFF + 15])
@@ -48,6 +77,11 @@ __device__ __forceinline__ void tmem_st_x16_nowait(uint32_t taddr, const uint32_
 template <int OFF, int N>
 __device__ __forceinline__ void tmem_st_x16_wait(uint32_t taddr, const uint32_t (&r)[N]) {
   static_assert(OFF + 16 <= N, "slice out of range");
+#ifdef ATTN_DEBUG_CHECKS
+  if (!debug_check(tmem_range_ok(taddr, 16))) {
+    return;
+  }
+#endif
   asm volatile(
     "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};\n\t"
     "tcgen05.wait::st.sync.aligned;\n"
@@ -57,6 +91,11 @@ __device__ __forceinline__ void tmem_st_x16_wait(uint32_t taddr, const uint32_t 
 template <int OFF, int N>
 __device__ __forceinline__ void tmem_st_x32_nowait(uint32_t taddr, const uint32_t (&r)[N]) {
   static_assert(OFF + 32 <= N, "slice out of range");
+#ifdef ATTN_DEBUG_CHECKS
+  if (!debug_check(tmem_range_ok(taddr, 32))) {
+    return;
+  }
+#endif
   asm volatile(
     "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};\n\t"
     :: "r"(taddr), "r"(r[OFF + 0]), "r"(r[OFF + 1]), "r"(r[OFF + 2]), "r"(r[OFF + 3]), "r"(r[OFF + 4]), "r"(r[OFF + 5]), "r"(r[OFF + 6]), "r"(r[OFF + 7]), "r"(r[OFF + 8]), "r"(r[OFF + 9]), "r"(r[OFF + 10]), "r"(r[OFF + 11]), "r"(r[OFF + 12]), "r"(r[OFF + 13]), "r"(r[OFF + 14]), "r"(r[OFF + 15]), "r"(r[OFF + 16]), "r"(r[OFF + 17]), "r"(r[OFF + 18]), "r"(r[OFF + 19]), "r"(r[OFF + 20]), "r"(r[OFF + 21]), "r"(r[OFF + 22]), "r"(r[OFF + 23]), "r"(r[OFF + 24]), "r"(r[OFF + 25]), "r"(r[OFF + 26]), "r"(r[OFF + 27]), "r"(r[OFF + 28]), "r"(r[OFF + 29]), "r"(r[OFF + 30]), "r"(r[OFF + 31])
@@ -65,6 +104,11 @@ __device__ __forceinline__ void tmem_st_x32_nowait(uint32_t taddr, const uint32_
 template <int OFF, int N>
 __device__ __forceinline__ void tmem_st_x32_wait(uint32_t taddr, const uint32_t (&r)[N]) {
   static_assert(OFF + 32 <= N, "slice out of range");
+#ifdef ATTN_DEBUG_CHECKS
+  if (!debug_check(tmem_range_ok(taddr, 32))) {
+    return;
+  }
+#endif
   asm volatile(
     "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};\n\t"
     "tcgen05.wait::st.sync.aligned;\n"
@@ -74,6 +118,11 @@ __device__ __forceinline__ void tmem_st_x32_wait(uint32_t taddr, const uint32_t 
 template <int OFF, int N>
 __device__ __forceinline__ void tmem_st_x64_nowait(uint32_t taddr, const uint32_t (&r)[N]) {
   static_assert(OFF + 64 <= N, "slice out of range");
+#ifdef ATTN_DEBUG_CHECKS
+  if (!debug_check(tmem_range_ok(taddr, 64))) {
+    return;
+  }
+#endif
   asm volatile(
     "tcgen05.st.sync.aligned.32x32b.x64.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63, %64};\n\t"
     :: "r"(taddr), "r"(r[OFF + 0]), "r"(r[OFF + 1]), "r"(r[OFF + 2]), "r"(r[OFF + 3]), "r"(r[OFF + 4]), "r"(r[OFF + 5]), "r"(r[OFF + 6]), "r"(r[OFF + 7]), "r"(r[OFF + 8]), "r"(r[OFF + 9]), "r"(r[OFF + 10]), "r"(r[OFF + 11]), "r"(r[OFF + 12]), "r"(r[OFF + 13]), "r"(r[OFF + 14]), "r"(r[OFF + 15]), "r"(r[OFF + 16]), "r"(r[OFF + 17]), "r"(r[OFF + 18]), "r"(r[OFF + 19]), "r"(r[OFF + 20]), "r"(r[OFF + 21]), "r"(r[OFF + 22]), "r"(r[OFF + 23]), "r"(r[OFF + 24]), "r"(r[OFF + 25]), "r"(r[OFF + 26]), "r"(r[OFF + 27]), "r"(r[OFF + 28]), "r"(r[OFF + 29]), "r"(r[OFF + 30]), "r"(r[OFF + 31]), "r"(r[OFF + 32]), "r"(r[OFF + 33]), "r"(r[OFF + 34]), "r"(r[OFF + 35]), "r"(r[OFF + 36]), "r"(r[OFF + 37]), "r"(r[OFF + 38]), "r"(r[OFF + 39]), "r"(r[OFF + 40]), "r"(r[OFF + 41]), "r"(r[OFF + 42]), "r"(r[OFF + 43]), "r"(r[OFF + 44]), "r"(r[OFF + 45]), "r"(r[OFF + 46]), "r"(r[OFF + 47]), "r"(r[OFF + 48]), "r"(r[OFF + 49]), "r"(r[OFF + 50]), "r"(r[OFF + 51]), "r"(r[OFF + 52]), "r"(r[OFF + 53]), "r"(r[OFF + 54]), "r"(r[OFF + 55]), "r"(r[OFF + 56]), "r"(r[OFF + 57]), "r"(r[OFF + 58]), "r"(r[OFF + 59]), "r"(r[OFF + 60]), "r"(r[OFF + 61]), "r"(r[OFF + 62]), "r"(r[OFF + 63])
@@ -82,6 +131,11 @@ __device__ __forceinline__ void tmem_st_x64_nowait(uint32_t taddr, const uint32_
 template <int OFF, int N>
 __device__ __forceinline__ void tmem_st_x64_wait(uint32_t taddr, const uint32_t (&r)[N]) {
   static_assert(OFF + 64 <= N, "slice out of range");
+#ifdef ATTN_DEBUG_CHECKS
+  if (!debug_check(tmem_range_ok(taddr, 64))) {
+    return;
+  }
+#endif
   asm volatile(
     "tcgen05.st.sync.aligned.32x32b.x64.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63, %64};\n\t"
     "tcgen05.wait::st.sync.aligned;\n"

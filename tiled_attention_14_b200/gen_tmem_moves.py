@@ -37,11 +37,26 @@ FOOTER = """
 """
 
 
+# In the debug build (ATTN_DEBUG_CHECKS) each move first checks its TMEM column range and lane
+# quarter (tmem_range_ok, ptx.cuh); a failed check is recorded and the move skipped (a load
+# then returns zeros).
+def _check(n: int, load: bool) -> str:
+    fill = f"    for (int i = 0; i < {n}; ++i) r[i] = 0u;\n" if load else ""
+    return (
+        "#ifdef ATTN_DEBUG_CHECKS\n"
+        f"  if (!debug_check(tmem_range_ok(taddr, {n}))) {{\n"
+        f"{fill}"
+        "    return;\n"
+        "  }\n"
+        "#endif\n")
+
+
 def _load(n: int) -> str:
     regs = ", ".join(f"%{i}" for i in range(n))
     outs = ", ".join(f'"=r"(r[{i}])' for i in range(n))
     return (
         f"__device__ __forceinline__ void tmem_ld_x{n}_wait(uint32_t taddr, uint32_t (&r)[{n}]) {{\n"
+        + _check(n, True) +
         f"  asm volatile(\n"
         f'    "tcgen05.ld.sync.aligned.32x32b.x{n}.b32 {{{regs}}}, [%{n}];\\n\\t"\n'
         f'    "tcgen05.wait::ld.sync.aligned;\\n"\n'
@@ -59,6 +74,7 @@ def _store(n: int, wait: bool) -> str:
         f"template <int OFF, int N>\n"
         f"__device__ __forceinline__ void {name}(uint32_t taddr, const uint32_t (&r)[N]) {{\n"
         f'  static_assert(OFF + {n} <= N, "slice out of range");\n'
+        + _check(n, False) +
         f"  asm volatile(\n"
         f'    "tcgen05.st.sync.aligned.32x32b.x{n}.b32 [%0], {{{regs}}};\\n\\t"\n'
         f"{wait_line}"
