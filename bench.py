@@ -608,6 +608,8 @@ def main():
                     help="time the device steps only (no e2e, sustained, per-config or CPU legs): "
                          "the command the ncu captures run")
     ap.add_argument("--heads", type=int, default=0, help="override H (smaller ncu captures)")
+    ap.add_argument("--backward", action="store_true",
+                    help="with --kernel-only: time attn_bwd (dQ, dK, dV) of the workload instead of the forward")
     ap.add_argument("--tau", type=float, default=None,
                     help="ablation builds only (TILED_ATTENTION_LIB=.../libattn_abl*.so): rescale threshold; "
                          "the line then reports the rescale counters")
@@ -650,6 +652,20 @@ def main():
     case = Case(ta, w, dev, seed=rank)
     stream = torch.cuda.current_stream(dev)
     quant_ms = case.quantize_ms() if w.fp8 else None
+    if args.backward:
+        if not args.kernel_only or w.fp8 or w.varlen:
+            ap.error("--backward needs --kernel-only and a BF16 batched workload")
+        case.step()
+        g = torch.Generator().manual_seed(1)
+        do = torch.randn(case.o.shape, generator=g).to(torch.bfloat16).to(dev)
+        grads = [torch.empty_like(t) for t in (case.q, case.k, case.v)]
+
+        def bwd_step():
+            ta.attn_bwd(case.q, case.k, case.v, case.o, case.lse, do, *grads, scale=w.scale,
+                        mask_kind=w.mask_kind, window=w.window, softcap=w.softcap, alibi_slopes=case.sl,
+                        doc_ids=case.doc)
+        case.step = bwd_step
+        case.launches_per_step = 3 + (1 if w.doc else 0)
 
     for _ in range(args.warmup):
         case.step()
@@ -685,7 +701,7 @@ def main():
     if ta.attn_get_status(stream) != 0:
         raise SystemExit("kernel status error in the timed region")
 
-    flops = algorithmic_flops(w)
+    flops = algorithmic_flops(w) * (2.5 if args.backward else 1.0)
     total_ms = max_over_ranks(total_ms, dist, dev)
     value = weak_scaling_value(flops, args.steps, world, total_ms)
     if ablation is not None:
@@ -699,7 +715,7 @@ def main():
         if rank == 0:
             line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
                     "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
-                    "config": workload_config(w), "kernel_only": True,
+                    "config": workload_config(w), "kernel_only": True, "backward": args.backward,
                     "gpu_launches": case.launches_per_step * args.steps}
             if ablation is not None:
                 line["ablation"] = ablation
