@@ -69,7 +69,9 @@ def test_profiled_traffic_is_gated_by_the_kernel_source_hash(tmp_path, monkeypat
     """A traffic figure is reported only while the kernel sources match the capture."""
     csrc = tmp_path / "tiled_attention_14_b200" / "csrc"
     csrc.mkdir(parents=True)
-    (csrc / "k.cuh").write_text("// kernel v1\n")
+    for f in bench.FWD_SOURCES:
+        (csrc / f).write_text("// source\n")
+    (csrc / "attn_fwd_kernel.cuh").write_text("// kernel v1\n")
     (tmp_path / "profiles").mkdir()
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     h = bench.kernel_source_hash()
@@ -77,5 +79,7 @@ def test_profiled_traffic_is_gated_by_the_kernel_source_hash(tmp_path, monkeypat
     (tmp_path / "profiles" / "traffic_causal.json").write_text(json.dumps(rec))
     assert bench.profiled_traffic("causal") == 123.0
     assert bench.profiled_traffic("long") is None              # no capture for this workload
-    (csrc / "k.cuh").write_text("// kernel v2\n")             # the kernel changed since
+    (csrc / "attn_bwd_kernel.cuh").write_text("// another kernel\n")   # not part of the forward
+    assert bench.profiled_traffic("causal") == 123.0
+    (csrc / "attn_fwd_kernel.cuh").write_text("// kernel v2\n")        # the kernel changed since
     assert bench.profiled_traffic("causal") is None

@@ -182,12 +182,13 @@ FwdParams make_params(void* o, float* lse, int B, int H, int Hkv, int Sq, int Sk
 }
 
 #ifndef ATTN_L2_GROUP_BYTES
-#define ATTN_L2_GROUP_BYTES (32ll << 20)
+#define ATTN_L2_GROUP_BYTES 0
 #endif
-// Causal longest-first order works through groups of heads whose K and V together take at
-// most ATTN_L2_GROUP_BYTES (a quarter of the 126 MB L2), so the K/V tiles that the CTAs in
-// flight re-read come from L2 rather than HBM.  Heads that share K/V (grouped-query) count
-// once per key/value head.  0 turns grouping off.
+// Causal longest-first order can work through groups of heads whose K and V together take at
+// most ATTN_L2_GROUP_BYTES, so that the K/V tiles the CTAs in flight re-read come from L2.
+// Measured on B200 with 32 MB groups it was much slower (causal B4 H16 S4096: 940 -> 712
+// TFLOP/s; FP8 causal 1101 -> 1004; grouped-query 1002 -> 914): the per-group longest-first
+// order leaves the CTAs' totals uneven.  0 (the default) keeps one group over all heads.
 int lpt_head_group(const FwdParams& p, int Sk, int D, int eb) {
   if (!p.lpt_qb_major || ATTN_L2_GROUP_BYTES <= 0) return 0;
   const long long kv_head = 2ll * Sk * D * eb;
@@ -376,130 +377,7 @@ int run_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* 
   return launch_fwd_d<64, false>(dev, tq, tk, tv, p, sc, al, stream);
 }
 
-// ---------------------------------------------------------------------------------------
-// Backward
-// ---------------------------------------------------------------------------------------
-template <int D, bool SOFTCAP, bool ALIBI>
-int launch_bwd_t(int dev, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                 const CUtensorMap& tdo, attn::BwdParams p, cudaStream_t stream) {
-  using C = attn::BwdCfg<D>;
-  auto ka = attn::attn_bwd_dkdv_kernel<D, SOFTCAP, ALIBI>;
-  auto kb = attn::attn_bwd_dq_kernel<D, SOFTCAP, ALIBI>;
-  static bool attr_set[kMaxDevices] = {};
-  if (!attr_set[dev]) {
-    if (cudaFuncSetAttribute(ka, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess ||
-        cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
-      return ATTN_ERR_CUDA;
-    attr_set[dev] = true;
-  }
-  const int sms = g_dev[dev].sms;
-  // dK / dV: one item per (b, key/value head, key tile)
-  p.num_items = p.B * p.Hkv * p.nkt;
-  int grid = p.num_items < sms ? p.num_items : sms;
-  ka<<<static_cast<unsigned>(grid), attn::kBwdThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, p);
-  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
-  // dQ: one item per (b, head, query tile)
-  p.num_items = p.B * p.H * p.nqt;
-  grid = p.num_items < sms ? p.num_items : sms;
-  kb<<<static_cast<unsigned>(grid), attn::kBwdThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, p);
-  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
-}
-
-template <int D>
-int launch_bwd_d(int dev, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                 const CUtensorMap& tdo, const attn::BwdParams& p, bool sc, bool al, cudaStream_t s) {
-  if (sc) return al ? launch_bwd_t<D, true, true>(dev, tq, tk, tv, tdo, p, s)
-                    : launch_bwd_t<D, true, false>(dev, tq, tk, tv, tdo, p, s);
-  return al ? launch_bwd_t<D, false, true>(dev, tq, tk, tv, tdo, p, s)
-            : launch_bwd_t<D, false, false>(dev, tq, tk, tv, tdo, p, s);
-}
-
-int run_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse, void* dq,
-            void* dk, void* dv, int B, int H, int Hkv, int Sq, int Sk, int D, float scale, int mask_kind, int window,
-            float softcap, const float* alibi, const int* doc_ids, cudaStream_t stream) {
-  int rc = check_common(q, k, v, o, lse, B, H, Sq, Sk, D, scale, mask_kind, window, softcap, alibi, doc_ids);
-  if (rc != ATTN_OK) return rc;
-  if (!dout || !dq || !dk || !dv) return ATTN_ERR_INVALID;
-  if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return ATTN_ERR_INVALID;
-  if (Hkv <= 0 || H % Hkv != 0) return ATTN_ERR_INVALID;
-  if ((mask_kind & ATTN_MASK_DOC) && B > 65535) return ATTN_ERR_INVALID;   // sorted-flag grid
-  const long long nqt = (Sq + 127) / 128, nkt = (Sk + 127) / 128;
-  if (static_cast<long long>(B) * H * nqt > 0x7fffffffLL || static_cast<long long>(B) * Hkv * nkt > 0x7fffffffLL)
-    return ATTN_ERR_INVALID;
-  int dev = 0;
-  if ((rc = current_device(&dev)) != ATTN_OK) return rc;
-
-  attn::BwdParams p;
-  std::memset(&p, 0, sizeof(p));
-  p.dq = static_cast<__nv_bfloat16*>(dq);
-  p.dk = static_cast<__nv_bfloat16*>(dk);
-  p.dv = static_cast<__nv_bfloat16*>(dv);
-  p.B = B;
-  p.H = H;
-  p.Hkv = Hkv;
-  p.group = H / Hkv;
-  p.Sq = Sq;
-  p.Sk = Sk;
-  p.nqt = static_cast<int>(nqt);
-  p.nkt = static_cast<int>(nkt);
-  p.Sq_pad = p.nqt * 128;
-  p.mask_kind = mask_kind;
-  const long long wmax = static_cast<long long>(Sq) + Sk;
-  p.window = (mask_kind & ATTN_MASK_WINDOW) ? static_cast<int>(window < wmax ? window : wmax) : 0;
-  const double log2e = 1.4426950408889634;
-  p.scale = scale;
-  p.scale_log2 = static_cast<float>(static_cast<double>(scale) * log2e);
-  if (softcap > 0.f) {
-    p.sc_in = static_cast<float>(static_cast<double>(scale) / softcap);
-    p.sc_out = static_cast<float>(static_cast<double>(softcap) * log2e);
-  }
-  p.alibi = alibi;
-  p.doc = (mask_kind & ATTN_MASK_DOC) ? doc_ids : nullptr;
-  p.lpt = ((mask_kind & ATTN_MASK_CAUSAL) && !(mask_kind & (ATTN_MASK_WINDOW | ATTN_MASK_DOC))) ? 1 : 0;
-  p.timeout_ns = static_cast<unsigned long long>(g_timeout_ms.load()) * 1000000ull;
-
-  CUtensorMap tq, tk, tv, tdo;
-  if (encode_map(&tq, q, false, B * H, Sq, D) != ATTN_OK || encode_map(&tdo, dout, false, B * H, Sq, D) != ATTN_OK ||
-      encode_map(&tk, k, false, B * Hkv, Sk, D) != ATTN_OK || encode_map(&tv, v, false, B * Hkv, Sk, D) != ATTN_OK)
-    return ATTN_ERR_CUDA;
-
-  // stream-ordered workspace: LSE * log2(e) and Dv padded to whole query tiles | sorted flags
-  const size_t rows = static_cast<size_t>(B) * H * p.Sq_pad;
-  const size_t ws_bytes = 2 * rows * sizeof(float) + ((static_cast<size_t>(B) * sizeof(int) + 15) & ~size_t(15));
-  void* ws = nullptr;
-  if (cudaMallocAsync(&ws, ws_bytes, stream) != cudaSuccess) return ATTN_ERR_NOMEM;
-  float* lse2 = static_cast<float*>(ws);
-  float* dvec = lse2 + rows;
-  int* sorted = reinterpret_cast<int*>(dvec + rows);
-  p.lse2 = lse2;
-  p.dvec = dvec;
-  {
-    long long blocks = (static_cast<long long>(rows) * 32 + attn::kPrepThreads - 1) / attn::kPrepThreads;
-    const long long cap = static_cast<long long>(g_dev[dev].sms) * 16;
-    if (blocks > cap) blocks = cap;
-    if (D == 128)
-      attn::attn_bwd_prep_kernel<128><<<static_cast<unsigned>(blocks), attn::kPrepThreads, 0, stream>>>(
-          static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, lse2, dvec, Sq,
-          p.Sq_pad, static_cast<long long>(rows));
-    else
-      attn::attn_bwd_prep_kernel<64><<<static_cast<unsigned>(blocks), attn::kPrepThreads, 0, stream>>>(
-          static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, lse2, dvec, Sq,
-          p.Sq_pad, static_cast<long long>(rows));
-    rc = cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
-  }
-  if (rc == ATTN_OK && p.doc != nullptr) {
-    attn::attn_doc_sorted_kernel<<<static_cast<unsigned>(B), attn::kSortedThreads, 0, stream>>>(p.doc, Sk, sorted);
-    rc = cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
-    p.doc_sorted = sorted;
-  }
-  if (rc == ATTN_OK) {
-    const bool sc = softcap > 0.f, al = alibi != nullptr;
-    rc = (D == 128) ? launch_bwd_d<128>(dev, tq, tk, tv, tdo, p, sc, al, stream)
-                    : launch_bwd_d<64>(dev, tq, tk, tv, tdo, p, sc, al, stream);
-  }
-  cudaFreeAsync(ws, stream);
-  return rc;
-}
+#include "attn_bwd_api.inc"
 
 }  // namespace
 
