@@ -22,11 +22,14 @@
 // dQ is computed apart from dK/dV (recomputing S and dP) instead of being summed across
 // CTAs, which is what keeps the result bit-reproducible.
 //
-// Each kernel: 6 warps — warps 0-3 compute (one thread per TMEM lane = one row of the
-// 128-row tile), warp 4 issues the TMA loads, one thread of warp 5 issues the MMAs.
+// Each kernel: 10 warps — warps 0-7 compute (two per TMEM lane quarter, one half of the 128
+// columns each), warp 8 issues the TMA loads, one thread of warp 9 issues the MMAs.
 // Tensor memory, dK/dV kernel: S^T | dP^T | dV | dK (P^T and dS^T in bf16 over the first
-// columns of S^T and dP^T); dQ kernel: S | dP | dQ (dS over dP).  Every wait is bounded as
-// in the forward kernel.
+// columns of S^T and dP^T); dQ kernel: S_a | S_b | dP | dQ (S double-buffered, dS in bf16
+// over the S it came from).  The hand-offs are split so that the tensor core works while the
+// compute warps do: in the dK/dV kernel dV and the next S^T run during the dS pass, dK and
+// the next dP^T during the next P pass; in the dQ kernel the next S is computed ahead.
+// Every wait is bounded as in the forward kernel.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
@@ -36,9 +39,13 @@
 
 namespace attn {
 
-constexpr int kBwdThreads = 192;
-constexpr int kBwdLoadWarp = 4;
-constexpr int kBwdMmaWarp = 5;
+// 10 warps: 0-7 compute (warps w and w+4 share the TMEM lane quarter w % 4 = 32 rows of the
+// tile and take one half of its 128 columns each), 8 issues the TMA loads, one thread of 9
+// issues the MMAs.
+constexpr int kBwdThreads = 320;
+constexpr int kBwdCompute = 256;
+constexpr int kBwdLoadWarp = 8;
+constexpr int kBwdMmaWarp = 9;
 
 struct BwdParams {
   __nv_bfloat16* dq;
@@ -72,7 +79,7 @@ struct BwdCfg {
   static constexpr int OFF_RING = 2 * TILE_BYTES;        // stage s: [OFF_RING + s*2*TILE, +TILE)
   static constexpr int OFF_ROWS = OFF_RING + NST * 2 * TILE_BYTES;   // NST x 1 KB (lse2, dvec)
   static constexpr int OFF_BAR = OFF_ROWS + NST * 1024;
-  static constexpr int NBAR = 16;
+  static constexpr int NBAR = 20;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   // At least 120 KB so that two CTAs never share an SM: each allocates all 512 TMEM
   // columns, and a second CTA on the SM would wait for the first one's to be freed.
@@ -80,6 +87,8 @@ struct BwdCfg {
   static constexpr int SMEM_BYTES = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t T_S = 0, T_DP = 128, T_ACC0 = 256, T_ACC1 = 256 + D;
+  // dQ kernel: two S buffers, dP, dQ
+  static constexpr uint32_t T_SB = 128, T_DPQ = 256, T_DQ = 384;
   static constexpr uint32_t IDESC_SS = make_idesc(1u, 128, 128, false);   // 128x128, both K-major
   static constexpr uint32_t IDESC_TS = make_idesc(1u, 128, D, true);      // A from TMEM, B MN-major
 };
@@ -210,6 +219,15 @@ __device__ __forceinline__ float bwd_modify(const BwdParams& p, float s, float s
   return t;
 }
 
+// Rendezvous of the 256 compute threads on an mbarrier of count 256 (one completion per use,
+// `parity` the use count's low bit): arrive, then a bounded wait, so that a thread whose
+// earlier wait ran out cannot leave the others waiting for ever.
+__device__ __forceinline__ bool compute_sync(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                             unsigned long long tmo) {
+  mbar_arrive(bar);
+  return __all_sync(0xffffffffu, wait_bounded(bar, parity, abort_flag, tmo));
+}
+
 // ---------------------------------------------------------------------------------------
 // dK / dV kernel
 // ---------------------------------------------------------------------------------------
@@ -263,10 +281,12 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
   const uint32_t sbase = (raw + 1023u) & ~1023u;
   uint8_t* sptr = smem_raw + (sbase - raw);
   auto BAR = [&](int i) -> uint32_t { return sbase + C::OFF_BAR + 8 * i; };
-  // barriers
+  // barriers: K/V of the item, the Q/dO ring, S^T and dP^T computed, P^T and dS^T written,
+  // the item's last MMAs, final drain
   constexpr int B_KVFULL = 0, B_KVEMPTY = 1, B_QFULL = 2, B_QEMPTY = 2 + C::NST, B_SFULL = 2 + 2 * C::NST,
-                B_PFULL = B_SFULL + 1, B_DONE = B_PFULL + 1, B_DRAIN = B_DONE + 1;
-  static_assert(B_DRAIN < C::NBAR, "barrier count");
+                B_DPFULL = B_SFULL + 1, B_PREADY = B_DPFULL + 1, B_DSREADY = B_PREADY + 1,
+                B_DONE = B_DSREADY + 1, B_DRAIN = B_DONE + 1, B_SYNC1 = B_DRAIN + 1, B_SYNC2 = B_SYNC1 + 1;
+  static_assert(B_SYNC2 < C::NBAR, "barrier count");
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sptr + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sptr + C::OFF_MISC + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -281,9 +301,13 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       mbar_init(BAR(B_QEMPTY + s), 1);
     }
     mbar_init(BAR(B_SFULL), 1);
-    mbar_init(BAR(B_PFULL), 128);
+    mbar_init(BAR(B_DPFULL), 1);
+    mbar_init(BAR(B_PREADY), kBwdCompute);
+    mbar_init(BAR(B_DSREADY), kBwdCompute);
     mbar_init(BAR(B_DONE), 1);
     mbar_init(BAR(B_DRAIN), 1);
+    mbar_init(BAR(B_SYNC1), kBwdCompute);
+    mbar_init(BAR(B_SYNC2), kBwdCompute);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -372,6 +396,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         for (int kk = 0; kk < 8; ++kk)
           mma_f16_ts(dst, a_tmem + kk * 8, b0 + ((kk * 16 * 128) >> 4), C::IDESC_TS, (acc || kk > 0) ? 1u : 0u);
       };
+      auto soff = [&](uint32_t idx) -> uint32_t { return ((idx % C::NST) * 2 * C::TILE_BYTES) >> 4; };
       uint32_t items = 0, cidx = 0, tcount = 0;
       bool ok = true;
       for (int r = 0; ok; ++r) {
@@ -380,24 +405,39 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         const KvItem it = make_kv_item(p, w);
         if (it.n == 0) continue;
         if (!wait_bounded(BAR(B_KVFULL), items & 1, abort_flag, tmo)) { ok = false; break; }
+        if (!wait_bounded(BAR(B_QFULL + cidx % C::NST), (cidx / C::NST) & 1, abort_flag, tmo)) { ok = false; break; }
         tc_fence_after();
+        // step 0: S^T = K Q^T and dP^T = V dO^T
+        ss(tS, dk_k, dring_k + soff(cidx));
+        mma_commit(BAR(B_SFULL));
+        ss(tDP, dv_k, dring_k + soff(cidx) + (C::TILE_BYTES >> 4));
+        mma_commit(BAR(B_DPFULL));
         for (int st = 0; st < it.n; ++st) {
-          const uint32_t slot = (cidx + st) % C::NST;
-          const uint32_t t = tcount + st;
-          if (!wait_bounded(BAR(B_QFULL + slot), ((cidx + st) / C::NST) & 1, abort_flag, tmo)) { ok = false; break; }
+          const uint32_t idx = cidx + st, t = tcount + st;
+          const bool more = st + 1 < it.n;
+          // dV += P^T dO once P^T is written; then the next S^T (over P^T: this thread's
+          // MMAs execute in issue order, so dV reads P^T first)
+          if (!wait_bounded(BAR(B_PREADY), t & 1, abort_flag, tmo)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t soff = (slot * 2 * C::TILE_BYTES) >> 4;
-          // S^T = K Q^T and dP^T = V dO^T (they overwrite P^T / dS^T of the previous step,
-          // which that step's dV / dK MMAs, issued earlier by this thread, read first)
-          ss(tS, dk_k, dring_k + soff);
-          ss(tDP, dv_k, dring_k + soff + (C::TILE_BYTES >> 4));
-          mma_commit(BAR(B_SFULL));
-          if (!wait_bounded(BAR(B_PFULL), t & 1, abort_flag, tmo)) { ok = false; break; }
+          ts(tDV, tS, dring_mn + soff(idx) + (C::TILE_BYTES >> 4), st > 0);
+          if (more) {
+            if (!wait_bounded(BAR(B_QFULL + (idx + 1) % C::NST), ((idx + 1) / C::NST) & 1, abort_flag, tmo)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            ss(tS, dk_k, dring_k + soff(idx + 1));
+            mma_commit(BAR(B_SFULL));
+          }
+          // dK += dS^T Q once dS^T is written; then the stage is free and the next dP^T
+          if (!wait_bounded(BAR(B_DSREADY), t & 1, abort_flag, tmo)) { ok = false; break; }
           tc_fence_after();
-          // dV += P^T dO,  dK += dS^T Q
-          ts(tDV, tS, dring_mn + soff + (C::TILE_BYTES >> 4), st > 0);
-          ts(tDK, tDP, dring_mn + soff, st > 0);
-          mma_commit(BAR(B_QEMPTY + slot));
+          ts(tDK, tDP, dring_mn + soff(idx), st > 0);
+          mma_commit(BAR(B_QEMPTY + idx % C::NST));
+          if (more) {
+            ss(tDP, dv_k, dring_k + soff(idx + 1) + (C::TILE_BYTES >> 4));
+            mma_commit(BAR(B_DPFULL));
+          }
         }
         if (!ok) break;
         mma_commit(BAR(B_KVEMPTY));
@@ -411,10 +451,11 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     }
   } else {
     // ------------------------------------------------------------------ compute warps
-    const int rloc = warp * 32 + lane;                       // key row within the tile (TMEM lane)
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const int quarter = warp & 3, half = warp >> 2;
+    const int rloc = quarter * 32 + lane;                    // key row within the tile (TMEM lane)
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t tS = tbase + C::T_S + lane_off, tDP = tbase + C::T_DP + lane_off;
-    const uint32_t tDV = tbase + C::T_ACC0 + lane_off, tDK = tbase + C::T_ACC1 + lane_off;
+    const int col0 = 64 * half;                              // this warp's query columns col0 .. col0+63
     const float* srows = reinterpret_cast<const float*>(sptr + C::OFF_ROWS);
     uint32_t tcount = 0, cidx = 0, items = 0;
     bool ok = true;
@@ -424,13 +465,10 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       const KvItem it = make_kv_item(p, w);
       const int j = it.nt * 128 + rloc;                      // key position
       if (it.n == 0) {
-        // no query row sees this key tile: dK = dV = 0
+        // no query row sees this key tile: dK = dV = 0 (warps 0-3 write dV, 4-7 dK)
         if (j < p.Sk) {
-          const size_t orow = (static_cast<size_t>(it.b * p.Hkv + it.kvh) * p.Sk + j) * D;
-          for (int c = 0; c < D; c += 8) {
-            *reinterpret_cast<uint4*>(p.dv + orow + c) = make_uint4(0u, 0u, 0u, 0u);
-            *reinterpret_cast<uint4*>(p.dk + orow + c) = make_uint4(0u, 0u, 0u, 0u);
-          }
+          __nv_bfloat16* dst = (half == 0 ? p.dv : p.dk) + (static_cast<size_t>(it.b * p.Hkv + it.kvh) * p.Sk + j) * D;
+          for (int c = 0; c < D; c += 8) *reinterpret_cast<uint4*>(dst + c) = make_uint4(0u, 0u, 0u, 0u);
         }
         continue;
       }
@@ -467,72 +505,92 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           break;
         }
         tc_fence_after();
-        const float* lse2 = srows + slot * 256;
-        const float* dvv = lse2 + 128;
-        // visible query columns of this key row within tile m
-        uint32_t vm[4];
-        interval_mask(ilo - m * 128, ihi - m * 128, vm);
-        const float rel0 = static_cast<float>(j - d - m * 128);    // j - i' for column 0
-        uint32_t pf[64];                                           // bf16 pairs of P * dt/ds
-        // pass 1: P^T = exp2(t - lse2) over S^T's first 64 columns
+        const float4* lse4 = reinterpret_cast<const float4*>(srows + slot * 256 + col0);
+        const float4* dvv4 = reinterpret_cast<const float4*>(srows + slot * 256 + 128 + col0);
+        // every query column of this warp's half visible to this key row (and no element test)
+        const int q0 = m * 128 + col0;
+        const bool full = __all_sync(0xffffffffu, !doc_elem && ilo <= q0 && ihi >= q0 + 63);
+        uint32_t vm[2];
+        {
+          uint32_t v4[4];
+          interval_mask(ilo - m * 128, ihi - m * 128, v4);
+          vm[0] = half ? v4[2] : v4[0];
+          vm[1] = half ? v4[3] : v4[1];
+        }
+        const float rel0 = static_cast<float>(j - d - q0);         // j - i' for this warp's column 0
+        // ---- pass 1: P^T = exp2(t - lse2), kept in registers as P * dt/ds for pass 2
+        uint32_t sa[32], sb[32];
+        auto sv = [&](int e) -> float { return __uint_as_float(e < 32 ? sa[e] : sb[e - 32]); };
+        tmem_ld_x32_wait(tS + col0, sa);
+        tmem_ld_x32_wait(tS + col0 + 32, sb);
+        // every warp has read its S^T columns before any P^T is written over them
+        if (!compute_sync(BAR(B_SYNC1), t & 1, abort_flag, tmo)) { ok = false; break; }
+        uint32_t pk[32], pf[32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t sv[32];
-          tmem_ld_x32_wait(tS + 32 * c, sv);
-          uint32_t pk[16];
+        for (int e4 = 0; e4 < 16; ++e4) {
+          const float4 l4 = lse4[e4];
+          const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const int col = 32 * c + e;
+          for (int u = 0; u < 4; u += 2) {
+            const int e = 4 * e4 + u;
             float f0, f1;
-            float t0 = bwd_modify<SOFTCAP, ALIBI>(p, __uint_as_float(sv[e]), slope_l2, rel0 - col, &f0);
-            float t1 = bwd_modify<SOFTCAP, ALIBI>(p, __uint_as_float(sv[e + 1]), slope_l2, rel0 - col - 1, &f1);
-            bool v0 = ((vm[col >> 5] >> (col & 31)) & 1u) != 0u;
-            bool v1 = ((vm[(col + 1) >> 5] >> ((col + 1) & 31)) & 1u) != 0u;
-            if (doc_elem) {
-              const int i0 = m * 128 + col;
-              v0 = v0 && i0 < p.Sq && __ldg(drow + min(i0, p.Sq - 1)) == doc_j;
-              v1 = v1 && i0 + 1 < p.Sq && __ldg(drow + min(i0 + 1, p.Sq - 1)) == doc_j;
+            const float t0 = bwd_modify<SOFTCAP, ALIBI>(p, sv(e), slope_l2, rel0 - e, &f0);
+            const float t1 = bwd_modify<SOFTCAP, ALIBI>(p, sv(e + 1), slope_l2, rel0 - e - 1, &f1);
+            float p0 = ex2_approx(t0 - lv[u]), p1 = ex2_approx(t1 - lv[u + 1]);
+            if (!full) {
+              bool v0 = ((vm[e >> 5] >> (e & 31)) & 1u) != 0u;
+              bool v1 = ((vm[(e + 1) >> 5] >> ((e + 1) & 31)) & 1u) != 0u;
+              if (doc_elem) {
+                const int i0 = q0 + e;
+                v0 = v0 && i0 < p.Sq && __ldg(drow + min(i0, p.Sq - 1)) == doc_j;
+                v1 = v1 && i0 + 1 < p.Sq && __ldg(drow + min(i0 + 1, p.Sq - 1)) == doc_j;
+              }
+              p0 = v0 ? p0 : 0.f;
+              p1 = v1 ? p1 : 0.f;
             }
-            const float p0 = v0 ? ex2_approx(t0 - lse2[col]) : 0.f;
-            const float p1 = v1 ? ex2_approx(t1 - lse2[col + 1]) : 0.f;
             pk[e >> 1] = pack_bf16x2(p0, p1);
-            pf[(32 * c + e) >> 1] = pack_bf16x2(p0 * f0, p1 * f1);
+            if constexpr (SOFTCAP) pf[e >> 1] = pack_bf16x2(p0 * f0, p1 * f1);
+            else pf[e >> 1] = pk[e >> 1];
           }
-          tmem_st_x16_nowait<0>(tS + 16 * c, pk);
         }
-        // pass 2: dS^T = (P dt/ds) (dP^T - Dv) over dP^T's first 64 columns
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t dv[32];
-          tmem_ld_x32_wait(tDP + 32 * c, dv);
-          uint32_t dk[16];
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const int col = 32 * c + e;
-            const float2 pp = unpack_bf16x2(pf[col >> 1]);
-            const float ds0 = pp.x * (__uint_as_float(dv[e]) - dvv[col]);
-            const float ds1 = pp.y * (__uint_as_float(dv[e + 1]) - dvv[col + 1]);
-            dk[e >> 1] = pack_bf16x2(ds0, ds1);
-          }
-          tmem_st_x16_nowait<0>(tDP + 16 * c, dk);
-        }
-        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        tmem_st_x32_wait<0>(tS + (col0 >> 1), pk);   // P^T: query pair (2c, 2c+1) in column c
         tc_fence_before();
-        mbar_arrive(BAR(B_PFULL));
+        mbar_arrive(BAR(B_PREADY));
+        // ---- pass 2: dS^T = (P dt/ds) (dP^T - Dv) over dP^T's first 64 columns
+        if (!__all_sync(0xffffffffu, wait_bounded(BAR(B_DPFULL), t & 1, abort_flag, tmo))) { ok = false; break; }
+        tc_fence_after();
+        tmem_ld_x32_wait(tDP + col0, sa);
+        tmem_ld_x32_wait(tDP + col0 + 32, sb);
+        // every warp has read its dP^T columns before any dS^T is written over them
+        if (!compute_sync(BAR(B_SYNC2), t & 1, abort_flag, tmo)) { ok = false; break; }
+        uint32_t dk[32];
+#pragma unroll
+        for (int e4 = 0; e4 < 16; ++e4) {
+          const float4 d4 = dvv4[e4];
+          const float dl[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+          for (int u = 0; u < 4; u += 2) {
+            const int e = 4 * e4 + u;
+            const float2 pp = unpack_bf16x2(pf[e >> 1]);
+            dk[e >> 1] = pack_bf16x2(pp.x * (sv(e) - dl[u]), pp.y * (sv(e + 1) - dl[u + 1]));
+          }
+        }
+        tmem_st_x32_wait<0>(tDP + (col0 >> 1), dk);
+        tc_fence_before();
+        mbar_arrive(BAR(B_DSREADY));
       }
       if (!__all_sync(0xffffffffu, ok && !*abort_flag)) {
         ok = false;
         break;
       }
-      // ---- epilogue: dV and scale * dK -> bf16
+      // ---- epilogue: warps 0-3 write dV, warps 4-7 write scale * dK (bf16)
       if (!__all_sync(0xffffffffu, wait_bounded(BAR(B_DONE), items & 1, abort_flag, tmo))) { ok = false; break; }
       tc_fence_after();
-      const size_t orow = (static_cast<size_t>(it.b * p.Hkv + it.kvh) * p.Sk + j) * D;
-#pragma unroll
-      for (int which = 0; which < 2; ++which) {
-        __nv_bfloat16* dst = (which == 0 ? p.dv : p.dk) + orow;
-        const float mul = which == 0 ? 1.f : p.scale;
-        const uint32_t src = which == 0 ? tDV : tDK;
+      {
+        const size_t orow = (static_cast<size_t>(it.b * p.Hkv + it.kvh) * p.Sk + j) * D;
+        __nv_bfloat16* dst = (half == 0 ? p.dv : p.dk) + orow;
+        const float mul = half == 0 ? 1.f : p.scale;
+        const uint32_t src = tbase + (half == 0 ? C::T_ACC0 : C::T_ACC1) + lane_off;
 #pragma unroll
         for (int ch = 0; ch < D / 32; ++ch) {
           uint32_t a[32];
@@ -585,7 +643,6 @@ __device__ __forceinline__ QItem make_q_item(const BwdParams& p, int w) {
   const int i0 = it.mt * 128, i1 = min(i0 + 127, p.Sq - 1);
   int c0 = max(keys_seen_by_row(p, i0).x, 0);
   int c1 = min(keys_seen_by_row(p, i1).y, p.Sk - 1);
-  if (p.mask_kind & 1) c0 = max(c0, 0);
   if (p.doc != nullptr && p.doc_sorted != nullptr && __ldg(p.doc_sorted + it.b)) {
     const int* drow = p.doc + static_cast<size_t>(it.b) * p.Sk;
     c0 = max(c0, doc_run(drow, p.Sk, i0).x);
@@ -612,9 +669,12 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   const uint32_t sbase = (raw + 1023u) & ~1023u;
   uint8_t* sptr = smem_raw + (sbase - raw);
   auto BAR = [&](int i) -> uint32_t { return sbase + C::OFF_BAR + 8 * i; };
+  // barriers: Q/dO of the item, the K/V ring, S computed (one per S buffer), dP computed,
+  // dS written, the item's last MMA, final drain, compute rendezvous
   constexpr int B_QFULL = 0, B_QEMPTY = 1, B_KVFULL = 2, B_KVEMPTY = 2 + C::NST, B_SFULL = 2 + 2 * C::NST,
-                B_PFULL = B_SFULL + 1, B_DONE = B_PFULL + 1, B_DRAIN = B_DONE + 1;
-  static_assert(B_DRAIN < C::NBAR, "barrier count");
+                B_DPFULL = B_SFULL + 2, B_DSREADY = B_DPFULL + 1, B_DONE = B_DSREADY + 1, B_DRAIN = B_DONE + 1,
+                B_SYNC = B_DRAIN + 1;
+  static_assert(B_SYNC < C::NBAR, "barrier count");
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sptr + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sptr + C::OFF_MISC + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -629,9 +689,12 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       mbar_init(BAR(B_KVEMPTY + s), 1);
     }
     mbar_init(BAR(B_SFULL), 1);
-    mbar_init(BAR(B_PFULL), 128);
+    mbar_init(BAR(B_SFULL + 1), 1);
+    mbar_init(BAR(B_DPFULL), 1);
+    mbar_init(BAR(B_DSREADY), kBwdCompute);
     mbar_init(BAR(B_DONE), 1);
     mbar_init(BAR(B_DRAIN), 1);
+    mbar_init(BAR(B_SYNC), kBwdCompute);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -693,7 +756,8 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   } else if (warp == kBwdMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t tS = tbase + C::T_S, tDP = tbase + C::T_DP, tDQ = tbase + C::T_ACC0;
+      const uint32_t tDP = tbase + C::T_DPQ, tDQ = tbase + C::T_DQ;
+      auto tSb = [&](uint32_t t) -> uint32_t { return tbase + ((t & 1u) ? C::T_SB : C::T_S); };
       const uint64_t dq_k = make_sdesc_sw128(sbase + C::OFF_A, 16, 1024);
       const uint64_t ddo_k = make_sdesc_sw128(sbase + C::OFF_B, 16, 1024);
       const uint64_t dring_k = make_sdesc_sw128(sbase + C::OFF_RING, 16, 1024);
@@ -706,6 +770,10 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           mma_f16_ss(dst, a0 + off, b0 + off, C::IDESC_SS, kk > 0);
         }
       };
+      auto soff = [&](uint32_t idx) -> uint32_t { return ((idx % C::NST) * 2 * C::TILE_BYTES) >> 4; };
+      auto kv_ready = [&](uint32_t idx) -> bool {
+        return wait_bounded(BAR(B_KVFULL + idx % C::NST), (idx / C::NST) & 1, abort_flag, tmo);
+      };
       uint32_t items = 0, cidx = 0, tcount = 0;
       bool ok = true;
       for (int r = 0; ok; ++r) {
@@ -713,24 +781,39 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         if (w >= p.num_items) break;
         const QItem it = make_q_item(p, w);
         if (it.n == 0) continue;
-        if (!wait_bounded(BAR(B_QFULL), items & 1, abort_flag, tmo)) { ok = false; break; }
+        if (!wait_bounded(BAR(B_QFULL), items & 1, abort_flag, tmo) || !kv_ready(cidx)) { ok = false; break; }
         tc_fence_after();
-        for (int st = 0; st < it.n; ++st) {
-          const uint32_t slot = (cidx + st) % C::NST;
-          const uint32_t t = tcount + st;
-          if (!wait_bounded(BAR(B_KVFULL + slot), ((cidx + st) / C::NST) & 1, abort_flag, tmo)) { ok = false; break; }
+        // S(0) = Q K^T and dP(0) = dO V^T; S(1) ahead into the other buffer
+        ss(tSb(tcount), dq_k, dring_k + soff(cidx));
+        mma_commit(BAR(B_SFULL + (tcount & 1)));
+        ss(tDP, ddo_k, dring_k + soff(cidx) + (C::TILE_BYTES >> 4));
+        mma_commit(BAR(B_DPFULL));
+        if (it.n > 1) {
+          if (!kv_ready(cidx + 1)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t soff = (slot * 2 * C::TILE_BYTES) >> 4;
-          ss(tS, dq_k, dring_k + soff);                                  // S = Q K^T
-          ss(tDP, ddo_k, dring_k + soff + (C::TILE_BYTES >> 4));         // dP = dO V^T
-          mma_commit(BAR(B_SFULL));
-          if (!wait_bounded(BAR(B_PFULL), t & 1, abort_flag, tmo)) { ok = false; break; }
+          ss(tSb(tcount + 1), dq_k, dring_k + soff(cidx + 1));
+          mma_commit(BAR(B_SFULL + ((tcount + 1) & 1)));
+        }
+        for (int st = 0; st < it.n; ++st) {
+          const uint32_t idx = cidx + st, t = tcount + st;
+          // dQ += dS K once dS is written (over S of this step)
+          if (!wait_bounded(BAR(B_DSREADY), t & 1, abort_flag, tmo)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)                                 // dQ += dS K
-            mma_f16_ts(tDQ, tDP + kk * 8, dring_mn + soff + ((kk * 16 * 128) >> 4), C::IDESC_TS,
+          for (int kk = 0; kk < 8; ++kk)
+            mma_f16_ts(tDQ, tSb(t) + kk * 8, dring_mn + soff(idx) + ((kk * 16 * 128) >> 4), C::IDESC_TS,
                        (st > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(BAR(B_KVEMPTY + slot));
+          mma_commit(BAR(B_KVEMPTY + idx % C::NST));
+          if (st + 1 < it.n) {   // dP of the next step (its K/V stage was waited for above)
+            ss(tDP, ddo_k, dring_k + soff(idx + 1) + (C::TILE_BYTES >> 4));
+            mma_commit(BAR(B_DPFULL));
+          }
+          if (st + 2 < it.n) {   // S two steps ahead, into the buffer dQ has just read
+            if (!kv_ready(idx + 2)) { ok = false; break; }
+            tc_fence_after();
+            ss(tSb(t), dq_k, dring_k + soff(idx + 2));
+            mma_commit(BAR(B_SFULL + (t & 1)));
+          }
         }
         if (!ok) break;
         mma_commit(BAR(B_QEMPTY));
@@ -744,10 +827,11 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     }
   } else {
     // ------------------------------------------------------------------ compute warps
-    const int rloc = warp * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t tS = tbase + C::T_S + lane_off, tDP = tbase + C::T_DP + lane_off;
-    const uint32_t tDQ = tbase + C::T_ACC0 + lane_off;
+    const int quarter = warp & 3, half = warp >> 2;
+    const int rloc = quarter * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tDP = tbase + C::T_DPQ + lane_off;
+    const int col0 = 64 * half;                              // this warp's key columns col0 .. col0+63
     uint32_t tcount = 0, items = 0;
     bool ok = true;
     for (int r = 0; ok; ++r) {
@@ -756,10 +840,10 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       const QItem it = make_q_item(p, w);
       const int i = it.mt * 128 + rloc;
       if (it.n == 0) {
-        // rows that see no key: dQ = 0
+        // rows that see no key: dQ = 0 (each half writes half of the row)
         if (i < p.Sq) {
-          __nv_bfloat16* dst = p.dq + (static_cast<size_t>(it.bh) * p.Sq + i) * D;
-          for (int c = 0; c < D; c += 8) *reinterpret_cast<uint4*>(dst + c) = make_uint4(0u, 0u, 0u, 0u);
+          __nv_bfloat16* dst = p.dq + (static_cast<size_t>(it.bh) * p.Sq + i) * D + half * (D / 2);
+          for (int c = 0; c < D / 2; c += 8) *reinterpret_cast<uint4*>(dst + c) = make_uint4(0u, 0u, 0u, 0u);
         }
         continue;
       }
@@ -789,42 +873,57 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       for (int st = 0; st < it.n; ++st) {
         const uint32_t t = tcount + st;
         const int kt = it.kt_lo + st;
-        if (!__all_sync(0xffffffffu, wait_bounded(BAR(B_SFULL), t & 1, abort_flag, tmo))) { ok = false; break; }
+        const uint32_t tS = tbase + ((t & 1u) ? C::T_SB : C::T_S) + lane_off;
+        if (!__all_sync(0xffffffffu, wait_bounded(BAR(B_SFULL + (t & 1)), (t >> 1) & 1, abort_flag, tmo) &&
+                                     wait_bounded(BAR(B_DPFULL), t & 1, abort_flag, tmo))) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        uint32_t vm[4];
-        interval_mask(jlo - kt * 128, jhi - kt * 128, vm);
-        const float rel0 = static_cast<float>(kt * 128 - ip);      // j - i' for column 0
+        const int c0 = kt * 128 + col0;
+        const bool full = __all_sync(0xffffffffu, !doc_elem && jlo <= c0 && jhi >= c0 + 63);
+        uint32_t vm[2];
+        {
+          uint32_t v4[4];
+          interval_mask(jlo - kt * 128, jhi - kt * 128, v4);
+          vm[0] = half ? v4[2] : v4[0];
+          vm[1] = half ? v4[3] : v4[1];
+        }
+        const float rel0 = static_cast<float>(c0 - ip);      // j - i' for this warp's column 0
+        uint32_t sa[32], sb[32];
+        tmem_ld_x32_wait(tS + col0, sa);
+        tmem_ld_x32_wait(tS + col0 + 32, sb);
+        // every warp has read its S columns before any dS is written over them
+        if (!compute_sync(BAR(B_SYNC), t & 1, abort_flag, tmo)) { ok = false; break; }
+        auto sv = [&](int e) -> float { return __uint_as_float(e < 32 ? sa[e] : sb[e - 32]); };
+        uint32_t dk[32];
+        uint32_t dq32[32];                                   // 32 columns of dP at a time
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t sv[32], dv[32];
-          tmem_ld_x32_wait(tS + 32 * c, sv);
-          tmem_ld_x32_wait(tDP + 32 * c, dv);
-          uint32_t dk[16];
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const int col = 32 * c + e;
-            float f0, f1;
-            const float t0 = bwd_modify<SOFTCAP, ALIBI>(p, __uint_as_float(sv[e]), slope_l2, rel0 + col, &f0);
-            const float t1 = bwd_modify<SOFTCAP, ALIBI>(p, __uint_as_float(sv[e + 1]), slope_l2, rel0 + col + 1, &f1);
-            bool v0 = ((vm[col >> 5] >> (col & 31)) & 1u) != 0u;
-            bool v1 = ((vm[(col + 1) >> 5] >> ((col + 1) & 31)) & 1u) != 0u;
+        for (int e = 0; e < 64; e += 2) {
+          if ((e & 31) == 0) tmem_ld_x32_wait(tDP + col0 + e, dq32);
+          auto dv = [&](int x) -> float { return __uint_as_float(dq32[x & 31]); };
+          float f0, f1;
+          const float t0 = bwd_modify<SOFTCAP, ALIBI>(p, sv(e), slope_l2, rel0 + e, &f0);
+          const float t1 = bwd_modify<SOFTCAP, ALIBI>(p, sv(e + 1), slope_l2, rel0 + e + 1, &f1);
+          float p0 = ex2_approx(t0 - lse2), p1 = ex2_approx(t1 - lse2);
+          if (!full) {
+            bool v0 = ((vm[e >> 5] >> (e & 31)) & 1u) != 0u;
+            bool v1 = ((vm[(e + 1) >> 5] >> ((e + 1) & 31)) & 1u) != 0u;
             if (doc_elem) {
-              const int j0 = kt * 128 + col;
+              const int j0 = c0 + e;
               v0 = v0 && j0 < p.Sk && __ldg(drow + min(j0, p.Sk - 1)) == doc_i;
               v1 = v1 && j0 + 1 < p.Sk && __ldg(drow + min(j0 + 1, p.Sk - 1)) == doc_i;
             }
-            const float p0 = v0 ? ex2_approx(t0 - lse2) : 0.f;
-            const float p1 = v1 ? ex2_approx(t1 - lse2) : 0.f;
-            // P * dt/ds rounded to bf16 first, as in the dK/dV kernel, so that both kernels
-            // use the same dS
-            const float2 pp = unpack_bf16x2(pack_bf16x2(p0 * f0, p1 * f1));
-            dk[e >> 1] = pack_bf16x2(pp.x * (__uint_as_float(dv[e]) - dvi), pp.y * (__uint_as_float(dv[e + 1]) - dvi));
+            p0 = v0 ? p0 : 0.f;
+            p1 = v1 ? p1 : 0.f;
           }
-          tmem_st_x16_nowait<0>(tDP + 16 * c, dk);
+          // P * dt/ds rounded to bf16 first, as in the dK/dV kernel, so that both use the same dS
+          const float2 pp = unpack_bf16x2(pack_bf16x2(p0 * f0, p1 * f1));
+          dk[e >> 1] = pack_bf16x2(pp.x * (dv(e) - dvi), pp.y * (dv(e + 1) - dvi));
         }
-        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        tmem_st_x32_wait<0>(tS + (col0 >> 1), dk);   // dS: key pair (2c, 2c+1) in column c
         tc_fence_before();
-        mbar_arrive(BAR(B_PFULL));
+        mbar_arrive(BAR(B_DSREADY));
       }
       if (!__all_sync(0xffffffffu, ok && !*abort_flag)) {
         ok = false;
@@ -832,17 +931,20 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       }
       if (!__all_sync(0xffffffffu, wait_bounded(BAR(B_DONE), items & 1, abort_flag, tmo))) { ok = false; break; }
       tc_fence_after();
+      // each half of the warps writes half of the dQ row (scale * dQ, bf16)
       __nv_bfloat16* dst = p.dq + (static_cast<size_t>(it.bh) * p.Sq + i) * D;
+      const uint32_t src = tbase + C::T_DQ + lane_off;
 #pragma unroll
-      for (int ch = 0; ch < D / 32; ++ch) {
+      for (int ch = 0; ch < D / 64; ++ch) {
+        const int cc = half * (D / 2) + ch * 32;
         uint32_t a[32];
-        tmem_ld_x32_wait(tDQ + ch * 32, a);
+        tmem_ld_x32_wait(src + cc, a);
         uint32_t wv[16];
 #pragma unroll
         for (int c = 0; c < 16; ++c)
           wv[c] = pack_bf16x2(__uint_as_float(a[2 * c]) * p.scale, __uint_as_float(a[2 * c + 1]) * p.scale);
         if (i < p.Sq) {
-          uint4* o4 = reinterpret_cast<uint4*>(dst + ch * 32);
+          uint4* o4 = reinterpret_cast<uint4*>(dst + cc);
 #pragma unroll
           for (int v = 0; v < 4; ++v) o4[v] = make_uint4(wv[4 * v], wv[4 * v + 1], wv[4 * v + 2], wv[4 * v + 3]);
         }
