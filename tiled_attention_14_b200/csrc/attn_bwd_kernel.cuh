@@ -228,6 +228,47 @@ __device__ __forceinline__ bool compute_sync(uint32_t bar, uint32_t parity, vola
   return __all_sync(0xffffffffu, wait_bounded(bar, parity, abort_flag, tmo));
 }
 
+// Visibility bits of 64 consecutive positions c0 .. c0+63 of a document-id row against one
+// id (unsorted ids: the element test, done once per step outside the element loops).
+__device__ __forceinline__ void doc_bits(const int* drow, int n, int c0, int id, uint32_t (&vm)[2]) {
+#pragma unroll
+  for (int w = 0; w < 2; ++w) {
+    uint32_t bits = 0u;
+    for (int c = 0; c < 32; ++c) {
+      const int x = c0 + 32 * w + c;
+      bits |= (x < n && __ldg(drow + min(x, n - 1)) == id) ? (1u << c) : 0u;
+    }
+    vm[w] &= bits;
+  }
+}
+
+// P (and P * dt/ds) for 64 scores of one row or column: p = 2^(t - lse), t the modified score;
+// with MASKED, positions whose bit in vm is clear get p = 0.  `lse_at(e)` gives the log2 LSE
+// of element e, `rel0 - sign * e` its relative position j - i'.  The loop is instantiated
+// once without and once with the mask so that the common, fully visible case runs a compact,
+// branch-free body.
+template <bool MASKED, bool SOFTCAP, bool ALIBI, int SIGN, typename LseAt>
+__device__ __forceinline__ void p_loop(const BwdParams& p, const uint32_t (&sa)[32], const uint32_t (&sb)[32],
+                                       const uint32_t (&vm)[2], float slope_l2, float rel0, LseAt lse_at,
+                                       uint32_t (&pk)[32], uint32_t (&pf)[32]) {
+#pragma unroll
+  for (int e = 0; e < 64; e += 2) {
+    const float s0 = __uint_as_float(e < 32 ? sa[e] : sb[e - 32]);
+    const float s1 = __uint_as_float(e + 1 < 32 ? sa[e + 1] : sb[e + 1 - 32]);
+    float f0, f1;
+    const float t0 = bwd_modify<SOFTCAP, ALIBI>(p, s0, slope_l2, rel0 + SIGN * e, &f0);
+    const float t1 = bwd_modify<SOFTCAP, ALIBI>(p, s1, slope_l2, rel0 + SIGN * (e + 1), &f1);
+    float p0 = ex2_approx(t0 - lse_at(e)), p1 = ex2_approx(t1 - lse_at(e + 1));
+    if constexpr (MASKED) {
+      p0 = ((vm[e >> 5] >> (e & 31)) & 1u) ? p0 : 0.f;
+      p1 = ((vm[(e + 1) >> 5] >> ((e + 1) & 31)) & 1u) ? p1 : 0.f;
+    }
+    pk[e >> 1] = pack_bf16x2(p0, p1);
+    if constexpr (SOFTCAP) pf[e >> 1] = pack_bf16x2(p0 * f0, p1 * f1);
+    else pf[e >> 1] = pk[e >> 1];
+  }
+}
+
 // ---------------------------------------------------------------------------------------
 // dK / dV kernel
 // ---------------------------------------------------------------------------------------
@@ -505,54 +546,30 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           break;
         }
         tc_fence_after();
-        const float4* lse4 = reinterpret_cast<const float4*>(srows + slot * 256 + col0);
+        const float* lse_row = srows + slot * 256 + col0;
         const float4* dvv4 = reinterpret_cast<const float4*>(srows + slot * 256 + 128 + col0);
         // every query column of this warp's half visible to this key row (and no element test)
         const int q0 = m * 128 + col0;
         const bool full = __all_sync(0xffffffffu, !doc_elem && ilo <= q0 && ihi >= q0 + 63);
-        uint32_t vm[2];
-        {
+        uint32_t vm[2] = {0xffffffffu, 0xffffffffu};
+        if (!full) {
           uint32_t v4[4];
           interval_mask(ilo - m * 128, ihi - m * 128, v4);
           vm[0] = half ? v4[2] : v4[0];
           vm[1] = half ? v4[3] : v4[1];
+          if (doc_elem) doc_bits(drow, p.Sq, q0, doc_j, vm);
         }
         const float rel0 = static_cast<float>(j - d - q0);         // j - i' for this warp's column 0
         // ---- pass 1: P^T = exp2(t - lse2), kept in registers as P * dt/ds for pass 2
         uint32_t sa[32], sb[32];
-        auto sv = [&](int e) -> float { return __uint_as_float(e < 32 ? sa[e] : sb[e - 32]); };
         tmem_ld_x32_wait(tS + col0, sa);
         tmem_ld_x32_wait(tS + col0 + 32, sb);
         // every warp has read its S^T columns before any P^T is written over them
         if (!compute_sync(BAR(B_SYNC1), t & 1, abort_flag, tmo)) { ok = false; break; }
         uint32_t pk[32], pf[32];
-#pragma unroll
-        for (int e4 = 0; e4 < 16; ++e4) {
-          const float4 l4 = lse4[e4];
-          const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-#pragma unroll
-          for (int u = 0; u < 4; u += 2) {
-            const int e = 4 * e4 + u;
-            float f0, f1;
-            const float t0 = bwd_modify<SOFTCAP, ALIBI>(p, sv(e), slope_l2, rel0 - e, &f0);
-            const float t1 = bwd_modify<SOFTCAP, ALIBI>(p, sv(e + 1), slope_l2, rel0 - e - 1, &f1);
-            float p0 = ex2_approx(t0 - lv[u]), p1 = ex2_approx(t1 - lv[u + 1]);
-            if (!full) {
-              bool v0 = ((vm[e >> 5] >> (e & 31)) & 1u) != 0u;
-              bool v1 = ((vm[(e + 1) >> 5] >> ((e + 1) & 31)) & 1u) != 0u;
-              if (doc_elem) {
-                const int i0 = q0 + e;
-                v0 = v0 && i0 < p.Sq && __ldg(drow + min(i0, p.Sq - 1)) == doc_j;
-                v1 = v1 && i0 + 1 < p.Sq && __ldg(drow + min(i0 + 1, p.Sq - 1)) == doc_j;
-              }
-              p0 = v0 ? p0 : 0.f;
-              p1 = v1 ? p1 : 0.f;
-            }
-            pk[e >> 1] = pack_bf16x2(p0, p1);
-            if constexpr (SOFTCAP) pf[e >> 1] = pack_bf16x2(p0 * f0, p1 * f1);
-            else pf[e >> 1] = pk[e >> 1];
-          }
-        }
+        auto lse_at = [&](int e) -> float { return lse_row[e]; };
+        if (full) p_loop<false, SOFTCAP, ALIBI, -1>(p, sa, sb, vm, slope_l2, rel0, lse_at, pk, pf);
+        else p_loop<true, SOFTCAP, ALIBI, -1>(p, sa, sb, vm, slope_l2, rel0, lse_at, pk, pf);
         tmem_st_x32_wait<0>(tS + (col0 >> 1), pk);   // P^T: query pair (2c, 2c+1) in column c
         tc_fence_before();
         mbar_arrive(BAR(B_PREADY));
@@ -572,7 +589,9 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           for (int u = 0; u < 4; u += 2) {
             const int e = 4 * e4 + u;
             const float2 pp = unpack_bf16x2(pf[e >> 1]);
-            dk[e >> 1] = pack_bf16x2(pp.x * (sv(e) - dl[u]), pp.y * (sv(e + 1) - dl[u + 1]));
+            const float x0 = __uint_as_float(e < 32 ? sa[e] : sb[e - 32]);
+            const float x1 = __uint_as_float(e + 1 < 32 ? sa[e + 1] : sb[e + 1 - 32]);
+            dk[e >> 1] = pack_bf16x2(pp.x * (x0 - dl[u]), pp.y * (x1 - dl[u + 1]));
           }
         }
         tmem_st_x32_wait<0>(tDP + (col0 >> 1), dk);
@@ -882,12 +901,13 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         tc_fence_after();
         const int c0 = kt * 128 + col0;
         const bool full = __all_sync(0xffffffffu, !doc_elem && jlo <= c0 && jhi >= c0 + 63);
-        uint32_t vm[2];
-        {
+        uint32_t vm[2] = {0xffffffffu, 0xffffffffu};
+        if (!full) {
           uint32_t v4[4];
           interval_mask(jlo - kt * 128, jhi - kt * 128, v4);
           vm[0] = half ? v4[2] : v4[0];
           vm[1] = half ? v4[3] : v4[1];
+          if (doc_elem) doc_bits(drow, p.Sk, c0, doc_i, vm);
         }
         const float rel0 = static_cast<float>(c0 - ip);      // j - i' for this warp's column 0
         uint32_t sa[32], sb[32];
@@ -895,31 +915,19 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         tmem_ld_x32_wait(tS + col0 + 32, sb);
         // every warp has read its S columns before any dS is written over them
         if (!compute_sync(BAR(B_SYNC), t & 1, abort_flag, tmo)) { ok = false; break; }
-        auto sv = [&](int e) -> float { return __uint_as_float(e < 32 ? sa[e] : sb[e - 32]); };
+        // P * dt/ds rounded to bf16 first, as in the dK/dV kernel, so that both use the same dS
+        uint32_t pk[32], pf[32];
+        auto lse_at = [&](int) -> float { return lse2; };
+        if (full) p_loop<false, SOFTCAP, ALIBI, 1>(p, sa, sb, vm, slope_l2, rel0, lse_at, pk, pf);
+        else p_loop<true, SOFTCAP, ALIBI, 1>(p, sa, sb, vm, slope_l2, rel0, lse_at, pk, pf);
         uint32_t dk[32];
         uint32_t dq32[32];                                   // 32 columns of dP at a time
 #pragma unroll
         for (int e = 0; e < 64; e += 2) {
           if ((e & 31) == 0) tmem_ld_x32_wait(tDP + col0 + e, dq32);
-          auto dv = [&](int x) -> float { return __uint_as_float(dq32[x & 31]); };
-          float f0, f1;
-          const float t0 = bwd_modify<SOFTCAP, ALIBI>(p, sv(e), slope_l2, rel0 + e, &f0);
-          const float t1 = bwd_modify<SOFTCAP, ALIBI>(p, sv(e + 1), slope_l2, rel0 + e + 1, &f1);
-          float p0 = ex2_approx(t0 - lse2), p1 = ex2_approx(t1 - lse2);
-          if (!full) {
-            bool v0 = ((vm[e >> 5] >> (e & 31)) & 1u) != 0u;
-            bool v1 = ((vm[(e + 1) >> 5] >> ((e + 1) & 31)) & 1u) != 0u;
-            if (doc_elem) {
-              const int j0 = c0 + e;
-              v0 = v0 && j0 < p.Sk && __ldg(drow + min(j0, p.Sk - 1)) == doc_i;
-              v1 = v1 && j0 + 1 < p.Sk && __ldg(drow + min(j0 + 1, p.Sk - 1)) == doc_i;
-            }
-            p0 = v0 ? p0 : 0.f;
-            p1 = v1 ? p1 : 0.f;
-          }
-          // P * dt/ds rounded to bf16 first, as in the dK/dV kernel, so that both use the same dS
-          const float2 pp = unpack_bf16x2(pack_bf16x2(p0 * f0, p1 * f1));
-          dk[e >> 1] = pack_bf16x2(pp.x * (dv(e) - dvi), pp.y * (dv(e + 1) - dvi));
+          const float2 pp = unpack_bf16x2(pf[e >> 1]);
+          dk[e >> 1] = pack_bf16x2(pp.x * (__uint_as_float(dq32[e & 31]) - dvi),
+                                   pp.y * (__uint_as_float(dq32[(e + 1) & 31]) - dvi));
         }
         tmem_st_x32_wait<0>(tS + (col0 >> 1), dk);   // dS: key pair (2c, 2c+1) in column c
         tc_fence_before();

@@ -57,11 +57,6 @@ static_assert(256 * kSoftmaxRegs + 128 * kControlRegs == kThreads * kLaunchRegs,
 constexpr int kLoadWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr float kTau = 8.0f;
-#ifndef ATTN_Q_PREFETCH
-#define ATTN_Q_PREFETCH 0
-#endif
-// Prefetch the next work item's query tiles into L2 during the current item.
-constexpr bool kQPrefetch = ATTN_Q_PREFETCH != 0;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kNegInf = -__builtin_huge_valf();
@@ -639,21 +634,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         ++qcount;
         for (int i = 0; i < it.n && ok; ++i) {
           const int kt = tile_kt(it, i);
-          if (kQPrefetch && i == (it.n > 1 ? 1 : 0)) {
-            // The next item's query tiles into L2 while this item runs, so that the loads at
-            // the item switch (issued once this item's last S MMAs are done) hit L2.
-            const int wn = sched_pos(r + 1, cta, G);
-            if (wn < p.num_items) {
-              const Item nx = make_item(p, wn);
-              if (nx.n > 0) {
-                for (int g = 0; g < 2; ++g) {
-                  const int qrow = nx.qb * 256 + 128 * g;
-                  const int qc1 = varlen ? nx.h : qrow, qc2 = varlen ? nx.q_off + qrow : nx.bh;
-                  for (int pn = 0; pn < C::NPANEL; ++pn) tma_prefetch_3d(&tm_q, pn * C::PANEL_COLS, qc1, qc2);
-                }
-              }
-            }
-          }
           for (int kv = 0; kv < 2; ++kv) {
             const uint32_t slot = lidx % C::NS;
             if (!wait_bounded(BAR(B_KVEMPTY + slot), ((lidx / C::NS) & 1) ^ 1, abort_flag, tmo)) {
