@@ -790,13 +790,21 @@ def main():
         }
         if quant_ms is not None:
             line["quantize_ms_per_tensor_set"] = quant_ms
+        if world == 1 and not args.no_per_config:
+            # each workload alone, before the seconds-long sustained loop heats the part
+            line["per_config"] = {}
+            for name in WORKLOADS:
+                time.sleep(0.5)
+                with ClockSampler(local, period_s=0.01) as cs:
+                    rec = per_config_record(ta, name, dev, peaks)
+                rec["clocks"] = cs.summary()
+                line["per_config"][name] = rec
+            with ClockSampler(local, period_s=0.01) as cs:
+                rec = bwd_record(ta, "causal", dev, peaks)
+            rec["clocks"] = cs.summary()
+            line["per_config"]["causal_backward"] = rec
         if world == 1:
             line["sustained"] = sustained_record(case, dev, peaks, local)
-        if world == 1 and not args.no_per_config:
-            del case
-            torch.cuda.empty_cache()
-            line["per_config"] = {name: per_config_record(ta, name, dev, peaks) for name in WORKLOADS}
-            line["per_config"]["causal_backward"] = bwd_record(ta, "causal", dev, peaks)
         if world == 1 and not args.no_cpu_baseline:
             f, dt, desc = oracle_sample(w, args.cpu_budget)
             line["cpu_baseline"] = {"value": f / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
