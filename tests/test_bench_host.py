@@ -61,7 +61,8 @@ def test_committed_traffic_files_are_well_formed():
         d = json.load(open(os.path.join(pdir, f)))
         assert f == f"traffic_{d['workload']}.json" and d["workload"] in bench.WORKLOADS
         assert len(d["kernel_source_hash"]) == 16
-        assert d["dram_bytes_read"] > 0 and d["dram_bytes_write"] > 0
+        # a small output can stay in L2 for the whole capture (no DRAM write)
+        assert d["dram_bytes_read"] > 0 and d["dram_bytes_write"] >= 0
         assert d["dram_bytes_per_launch"] == d["dram_bytes_read"] + d["dram_bytes_write"]
 
 
