@@ -117,6 +117,24 @@ ATTN_API int attn_fwd_gqa(const void* q, const void* k, const void* v, void* o, 
                           const float* alibi_slopes, const int* doc_ids, void* stream);
 
 /*
+ * attn_fwd_pair — attn_fwd_gqa computed by the kernel that runs each 256-row query block on a
+ * cluster of two CTAs on two SMs: the pair MMA (tcgen05 cta_group::2, M = 256) with each CTA
+ * holding 128 query rows, half of every K/V tile and two S buffers in its tensor memory, so
+ * that S of the next key tile overlaps the softmax of this one.  The page "Hardware-Aware FP4
+ * FlashAttention-4" (paragraph on on-chip storage) names the full on-chip storage that keeps
+ * stages from overlapping; the FlexAttention page names the 256x128 Blackwell tile (section
+ * "Aktuelle Einschränkungen").  BF16 with D = 128 only (other D: ATTN_ERR_INVALID); same
+ * arguments, layouts, masks and results (within the same tolerance) as attn_fwd_gqa.
+ * Measured on B200 it is slower than attn_fwd (about 0.8x), which is why attn_fwd does not
+ * use it; it is kept as a tested alternative.  Launched as 2-CTA clusters; every wait is
+ * bounded as in attn_fwd.
+ */
+ATTN_API int attn_fwd_pair(const void* q, const void* k, const void* v, void* o, float* lse,
+                           int B, int H, int H_kv, int Sq, int Sk, int D, float scale,
+                           int mask_kind, int window, float softcap,
+                           const float* alibi_slopes, const int* doc_ids, void* stream);
+
+/*
  * attn_fwd_varlen — attention over packed variable-length sequences, without padding
  * (page "FlashAttention 4: ...", section "Συμβατότητα και τρέχουσα κατάσταση").
  * Sequence s owns query tokens cu_seqlens_q[s] .. cu_seqlens_q[s+1]-1 and key tokens

@@ -54,6 +54,11 @@ def test_bad_arguments_rejected(kw):
 
 def test_bad_arguments_other_entry_points():
     lib = _lib.load()
+    # the pair kernel takes BF16 with D = 128 only
+    assert lib.attn_fwd_pair(A, A, A, A, A, 1, 1, 1, 128, 128, 64, 0.1, 0, 0, 0.0, None, None, None) == \
+        _lib.ATTN_ERR_INVALID
+    assert lib.attn_fwd_pair(A, A, A, A, A, 1, 2, 3, 128, 128, 128, 0.1, 0, 0, 0.0, None, None, None) == \
+        _lib.ATTN_ERR_INVALID
     assert lib.attn_quantize_e4m3(A, A, A, 1, 1, 128, 96 + 8, None) == _lib.ATTN_ERR_INVALID
     assert lib.attn_quantize_e4m3(None, A, A, 1, 1, 128, 64, None) == _lib.ATTN_ERR_INVALID
     assert lib.attn_tile_map_build(None, A, 1, 128, 128, 0, 0, None, None) == _lib.ATTN_ERR_INVALID

@@ -33,3 +33,28 @@ def test_skipped_signal_times_out_and_context_survives():
     assert ta.attn_get_status() == _lib.ATTN_OK
     O, L, E = oracle_eav(q, k, v, 1.0 / 128 ** 0.5, MASK_CAUSAL)
     compare(o, lse, O, L, eav=E)
+
+
+def test_pair_kernel_skipped_signal_times_out_and_context_survives():
+    """The same hook in the pair kernel: the odd CTA's first softmax warp skips its first
+    P-ready arrival on the even CTA's barrier; the MMA issuer's wait runs out, the other CTA's
+    waits run out in turn, both CTAs still meet at their final cluster barrier and free the
+    pair's tensor memory."""
+    import tiled_attention_14_b200 as ta
+    from tiled_attention_14_b200 import _lib
+    lib = _lib.load()
+    q, k, v = make_qkv(1, 2, 640, 640, 128, seed=42)
+    qd, kd, vd = to_dev(q, k, v)
+    assert ta.attn_get_status() == _lib.ATTN_OK
+    lib.attn_debug_set_fault(1, 200)
+    try:
+        ta.attn_fwd_pair(qd, kd, vd, mask_kind=MASK_CAUSAL)
+        assert ta.attn_get_status() == _lib.ATTN_ERR_TIMEOUT
+    finally:
+        lib.attn_debug_set_fault(0, 1000)
+    assert ta.attn_get_status() == _lib.ATTN_OK
+    o, lse = ta.attn_fwd_pair(qd, kd, vd, mask_kind=MASK_CAUSAL)
+    torch.cuda.synchronize()
+    assert ta.attn_get_status() == _lib.ATTN_OK
+    O, L, E = oracle_eav(q, k, v, 1.0 / 128 ** 0.5, MASK_CAUSAL)
+    compare(o, lse, O, L, eav=E)

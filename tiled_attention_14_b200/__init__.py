@@ -13,7 +13,7 @@ import torch
 from ._lib import (ATTN_ERR_TIMEOUT, ATTN_OK, MASK_CAUSAL, MASK_DOC, MASK_NONE, MASK_WINDOW,
                    AttnError, check, load)
 
-__all__ = ["attn_fwd", "attn_bwd", "attn_fwd_varlen", "attn_fwd_noalloc", "attn_fwd_with_map", "attn_fwd_fp8", "attn_quantize_e4m3",
+__all__ = ["attn_fwd", "attn_fwd_pair", "attn_bwd", "attn_fwd_varlen", "attn_fwd_noalloc", "attn_fwd_with_map", "attn_fwd_fp8", "attn_quantize_e4m3",
            "attn_tile_map_build", "attn_get_status", "attn_shutdown", "tile_map_shape",
            "AttnError", "MASK_NONE", "MASK_CAUSAL", "MASK_WINDOW", "MASK_DOC"]
 
@@ -107,6 +107,25 @@ def attn_fwd(q, k, v, o=None, lse=None, scale=None, mask_kind=MASK_NONE, window=
                               int(mask_kind), int(window), float(softcap), _ptr(alibi_slopes), _ptr(doc_ids),
                               _stream(stream))
         check(rc, "attn_fwd_gqa")
+    return o, lse
+
+
+def attn_fwd_pair(q, k, v, o=None, lse=None, scale=None, mask_kind=MASK_NONE, window=0, softcap=0.0,
+                  alibi_slopes=None, doc_ids=None, stream=None):
+    """attn_fwd computed on pairs of SMs (2-CTA clusters, tcgen05 cta_group::2); BF16, D = 128.
+    Same arguments and results as attn_fwd (grouped heads included); slower than attn_fwd on
+    B200, kept as a tested alternative."""
+    lib = load()
+    B, H, Hkv, Sq, Sk, D = _check_qkv(q, k, v, torch.bfloat16, gqa=True)
+    if D != 128:
+        raise ValueError("attn_fwd_pair needs D = 128")
+    _check_mods(q, H, B, Sk, alibi_slopes, doc_ids)
+    o, lse = _out(q, o, lse)
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    rc = lib.attn_fwd_pair(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Hkv, Sq, Sk, D, float(scale),
+                           int(mask_kind), int(window), float(softcap), _ptr(alibi_slopes), _ptr(doc_ids),
+                           _stream(stream))
+    check(rc, "attn_fwd_pair")
     return o, lse
 
 

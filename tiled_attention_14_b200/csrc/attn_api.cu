@@ -18,6 +18,7 @@
 #endif
 #include "attn_bwd_kernel.cuh"
 #include "attn_fwd_kernel.cuh"
+#include "attn_fwd_pair_kernel.cuh"
 #include "quant_kernel.cuh"
 #include "tile_map_kernel.cuh"
 
@@ -91,10 +92,10 @@ int check_common(const void* q, const void* k, const void* v, const void* o, con
 
 // Packed token-major tensor [T, Hx, D]: map (D, Hx, T), box 64 or 128 columns x 1 head x
 // 128 tokens, so a box lands in shared memory exactly as a batched tile does.
-int encode_map_thd(CUtensorMap* map, const void* ptr, int Hx, int T, int D) {
+int encode_map_thd(CUtensorMap* map, const void* ptr, int Hx, int T, int D, int box_tokens = 128) {
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Hx), static_cast<cuuint64_t>(T)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(Hx) * D * 2};
-  cuuint32_t box[3] = {64u, 1u, 128u};
+  cuuint32_t box[3] = {64u, 1u, static_cast<cuuint32_t>(box_tokens)};
   cuuint32_t estr[3] = {1u, 1u, 1u};
   const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
                               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -102,11 +103,11 @@ int encode_map_thd(CUtensorMap* map, const void* ptr, int Hx, int T, int D) {
   return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
-int encode_map(CUtensorMap* map, const void* ptr, bool fp8, int BH, int S, int D) {
+int encode_map(CUtensorMap* map, const void* ptr, bool fp8, int BH, int S, int D, int box_rows = 128) {
   const int eb = fp8 ? 1 : 2;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(S), static_cast<cuuint64_t>(BH)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * eb, static_cast<cuuint64_t>(S) * D * eb};
-  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / eb), 128u, 1u};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / eb), static_cast<cuuint32_t>(box_rows), 1u};
   cuuint32_t estr[3] = {1u, 1u, 1u};
   const CUresult r = g_encode(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
                               const_cast<void*>(ptr), dims, strides, box, estr,
@@ -142,6 +143,60 @@ int launch_fwd_d(int dev, const CUtensorMap& tq, const CUtensorMap& tk, const CU
   }
   return alibi ? launch_fwd_t<D, FP8, false, true>(dev, tq, tk, tv, p, s)
                : launch_fwd_t<D, FP8, false, false>(dev, tq, tk, tv, p, s);
+}
+
+// The pair kernel (attn_fwd_pair_kernel, BF16, D = 128) runs through attn_fwd_pair only:
+// measured on B200 it reaches about 80 % of the single-CTA kernel's rate (causal B4 H16 S4096
+// 738 against 925 TFLOP/s, non-causal B1 H32 S32768 885 against 1055), so the other entry
+// points keep the single-CTA kernel.  ATTN_PAIR_SPLIT softmax warps share each query row (2:
+// 64 keys each; 4 measured slower).
+#ifndef ATTN_PAIR_SPLIT
+#define ATTN_PAIR_SPLIT 2
+#endif
+
+template <bool SOFTCAP, bool ALIBI>
+int launch_pair_t(int dev, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
+                  cudaStream_t stream) {
+  using C = attn::CfgPair<ATTN_PAIR_SPLIT>;
+  auto kern = attn::attn_fwd_pair_kernel<ATTN_PAIR_SPLIT, SOFTCAP, ALIBI>;
+  static bool attr_set[kMaxDevices] = {};
+  static int clusters[kMaxDevices] = {};
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    attr_set[dev] = true;
+  }
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(C::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (clusters[dev] == 0) {
+    // Persistent grid: as many pairs as can be resident at once (one CTA per SM; SMs that
+    // cannot be paired inside their GPC stay idle).
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * (g_dev[dev].sms / 2)), 1, 1);
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) return ATTN_ERR_CUDA;
+    clusters[dev] = n;
+  }
+  const int pairs = p.num_items < clusters[dev] ? p.num_items : clusters[dev];
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs), 1, 1);
+  if (cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, p) != cudaSuccess) return ATTN_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+int launch_pair(int dev, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
+                bool softcap, bool alibi, cudaStream_t s) {
+  if (softcap) {
+    return alibi ? launch_pair_t<true, true>(dev, tq, tk, tv, p, s) : launch_pair_t<true, false>(dev, tq, tk, tv, p, s);
+  }
+  return alibi ? launch_pair_t<false, true>(dev, tq, tk, tv, p, s) : launch_pair_t<false, false>(dev, tq, tk, tv, p, s);
 }
 
 // Fills the parameter block shared by the BF16 and FP8 paths.
@@ -225,11 +280,12 @@ size_t ws_bytes_for_map(int B, int Sq, int Sk) {
 int run_fwd(bool fp8, const void* q, const void* k, const void* v, const float* qs, const float* ks,
             const float* vs, void* o, float* lse, int B, int H, int Hkv, int Sq, int Sk, int D, float scale,
             int mask_kind, int window, float softcap, const float* alibi, const int* doc_ids,
-            const int* counts, const uint32_t* entries, cudaStream_t stream) {
+            const int* counts, const uint32_t* entries, cudaStream_t stream, bool pair = false) {
   int rc = check_common(q, k, v, o, lse, B, H, Sq, Sk, D, scale, mask_kind, window, softcap, alibi, doc_ids);
   if (rc != ATTN_OK) return rc;
   if (Hkv <= 0 || H % Hkv != 0) return ATTN_ERR_INVALID;
   if (fp8 && (D != 128 || !qs || !ks || !vs)) return ATTN_ERR_INVALID;
+  if (pair && (fp8 || D != 128)) return ATTN_ERR_INVALID;
   if ((counts == nullptr) != (entries == nullptr)) return ATTN_ERR_INVALID;
   // the tile-map build launches one grid row per batch entry (grid.y <= 65535)
   if (counts == nullptr && (mask_kind & ATTN_MASK_DOC) && B > 65535) return ATTN_ERR_INVALID;
@@ -246,7 +302,8 @@ int run_fwd(bool fp8, const void* q, const void* k, const void* v, const float* 
   }
   p.lpt_heads = lpt_head_group(p, Sk, D, fp8 ? 1 : 2);
   CUtensorMap tq, tk, tv;
-  if (encode_map(&tq, q, fp8, B * H, Sq, D) != ATTN_OK || encode_map(&tk, k, fp8, B * Hkv, Sk, D) != ATTN_OK ||
+  if (encode_map(&tq, q, fp8, B * H, Sq, D) != ATTN_OK ||
+      encode_map(&tk, k, fp8, B * Hkv, Sk, D, pair ? 64 : 128) != ATTN_OK ||
       encode_map(&tv, v, fp8, B * Hkv, Sk, D) != ATTN_OK)
     return ATTN_ERR_CUDA;
 
@@ -270,6 +327,7 @@ int run_fwd(bool fp8, const void* q, const void* k, const void* v, const float* 
   p.map_entries = entries;
   const bool sc = softcap > 0.f, al = alibi != nullptr;
   if (fp8) rc = launch_fwd_d<128, true>(dev, tq, tk, tv, p, sc, al, stream);
+  else if (pair) rc = launch_pair(dev, tq, tk, tv, p, sc, al, stream);
   else if (D == 128) rc = launch_fwd_d<128, false>(dev, tq, tk, tv, p, sc, al, stream);
   else rc = launch_fwd_d<64, false>(dev, tq, tk, tv, p, sc, al, stream);
   if (ws) cudaFreeAsync(ws, stream);
@@ -395,6 +453,13 @@ int attn_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* ls
                  const float* alibi_slopes, const int* doc_ids, void* stream) {
   return run_fwd(false, q, k, v, nullptr, nullptr, nullptr, o, lse, B, H, H_kv, Sq, Sk, D, scale, mask_kind,
                  window, softcap, alibi_slopes, doc_ids, nullptr, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+int attn_fwd_pair(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv,
+                  int Sq, int Sk, int D, float scale, int mask_kind, int window, float softcap,
+                  const float* alibi_slopes, const int* doc_ids, void* stream) {
+  return run_fwd(false, q, k, v, nullptr, nullptr, nullptr, o, lse, B, H, H_kv, Sq, Sk, D, scale, mask_kind,
+                 window, softcap, alibi_slopes, doc_ids, nullptr, nullptr, static_cast<cudaStream_t>(stream), true);
 }
 
 int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu_seqlens_q,
