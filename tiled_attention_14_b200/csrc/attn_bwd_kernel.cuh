@@ -25,10 +25,12 @@
 // Each kernel: 10 warps — warps 0-7 compute (two per TMEM lane quarter, one half of the 128
 // columns each), warp 8 issues the TMA loads, one thread of warp 9 issues the MMAs.
 // Tensor memory, dK/dV kernel: S^T | dP^T | dV | dK (P^T and dS^T in bf16 over the first
-// columns of S^T and dP^T); dQ kernel: S_a | S_b | dP | dQ (S double-buffered, dS in bf16
-// over the S it came from).  The hand-offs are split so that the tensor core works while the
+// columns of S^T and dP^T); dQ kernel: S | dP_0 | dP_1 | dQ (dP double-buffered, dS in bf16
+// over the dP it came from).  The hand-offs are split so that the tensor core works while the
 // compute warps do: in the dK/dV kernel dV and the next S^T run during the dS pass, dK and
-// the next dP^T during the next P pass; in the dQ kernel the next S is computed ahead.
+// the next dP^T during the next P pass; in the dQ kernel the next S is computed as soon as
+// this step's S has been read and the dP two steps ahead right after dQ, so that a step never
+// waits for the tensor core.
 // Every wait is bounded as in the forward kernel.
 #pragma once
 #include <cstdint>
@@ -87,8 +89,19 @@ struct BwdCfg {
   static constexpr int SMEM_BYTES = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t T_S = 0, T_DP = 128, T_ACC0 = 256, T_ACC1 = 256 + D;
-  // dQ kernel: two S buffers, dP, dQ
-  static constexpr uint32_t T_SB = 128, T_DPQ = 256, T_DQ = 384;
+  // dQ kernel: S, two dP buffers (dS is written over the dP it came from), dQ
+  static constexpr uint32_t T_DP0 = 128, T_DP1 = 256, T_DQ = 384;
+  // dQ kernel shared memory: Q | dO | K ring | V ring.  K is read by S one step ahead and by
+  // dQ at the end of its step; V only by dP, two steps ahead: so K gets three slots and V two,
+  // which lets every slot be reloaded a full step before it is needed.
+  static constexpr int DQ_NK = 3, DQ_NV = 2;
+  static constexpr int DQ_OFF_K = 2 * TILE_BYTES;
+  static constexpr int DQ_OFF_V = DQ_OFF_K + DQ_NK * TILE_BYTES;
+  static constexpr int DQ_OFF_BAR = DQ_OFF_V + DQ_NV * TILE_BYTES;
+  static constexpr int DQ_OFF_MISC = DQ_OFF_BAR + NBAR * 8;
+  static constexpr int DQ_SMEM_USED = DQ_OFF_MISC + 16 + 1024;
+  static constexpr int DQ_SMEM_BYTES = DQ_SMEM_USED > 120 * 1024 ? DQ_SMEM_USED : 120 * 1024;
+  static_assert(DQ_SMEM_BYTES <= 227 * 1024, "dQ kernel shared memory");
   static constexpr uint32_t IDESC_SS = make_idesc(1u, 128, 128, false);   // 128x128, both K-major
   static constexpr uint32_t IDESC_TS = make_idesc(1u, 128, D, true);      // A from TMEM, B MN-major
 };
@@ -687,15 +700,17 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
   uint8_t* sptr = smem_raw + (sbase - raw);
-  auto BAR = [&](int i) -> uint32_t { return sbase + C::OFF_BAR + 8 * i; };
-  // barriers: Q/dO of the item, the K/V ring, S computed (one per S buffer), dP computed,
-  // dS written, the item's last MMA, final drain, compute rendezvous
-  constexpr int B_QFULL = 0, B_QEMPTY = 1, B_KVFULL = 2, B_KVEMPTY = 2 + C::NST, B_SFULL = 2 + 2 * C::NST,
-                B_DPFULL = B_SFULL + 2, B_DSREADY = B_DPFULL + 1, B_DONE = B_DSREADY + 1, B_DRAIN = B_DONE + 1,
-                B_SYNC = B_DRAIN + 1;
+  auto BAR = [&](int i) -> uint32_t { return sbase + C::DQ_OFF_BAR + 8 * i; };
+  // barriers: Q/dO of the item, the K ring, the V ring, S computed, S read by the compute
+  // warps, dP computed (one per dP buffer), dS written, the item's last MMA, final drain,
+  // compute rendezvous
+  constexpr int NK = C::DQ_NK, NV = C::DQ_NV;
+  constexpr int B_QFULL = 0, B_QEMPTY = 1, B_KFULL = 2, B_KEMPTY = 2 + NK, B_VFULL = 2 + 2 * NK,
+                B_VEMPTY = B_VFULL + NV, B_SFULL = B_VEMPTY + NV, B_SFREE = B_SFULL + 1, B_DPFULL = B_SFREE + 1,
+                B_DSREADY = B_DPFULL + 2, B_DONE = B_DSREADY + 1, B_DRAIN = B_DONE + 1, B_SYNC = B_DRAIN + 1;
   static_assert(B_SYNC < C::NBAR, "barrier count");
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sptr + C::OFF_MISC);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(sptr + C::OFF_MISC + 4);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sptr + C::DQ_OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sptr + C::DQ_OFF_MISC + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = gridDim.x, cta = blockIdx.x;
   const unsigned long long tmo = p.timeout_ns;
@@ -703,13 +718,18 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   if (threadIdx.x == 0) {
     mbar_init(BAR(B_QFULL), 1);
     mbar_init(BAR(B_QEMPTY), 1);
-    for (int s = 0; s < C::NST; ++s) {
-      mbar_init(BAR(B_KVFULL + s), 1);
-      mbar_init(BAR(B_KVEMPTY + s), 1);
+    for (int s = 0; s < NK; ++s) {
+      mbar_init(BAR(B_KFULL + s), 1);
+      mbar_init(BAR(B_KEMPTY + s), 1);
+    }
+    for (int s = 0; s < NV; ++s) {
+      mbar_init(BAR(B_VFULL + s), 1);
+      mbar_init(BAR(B_VEMPTY + s), 1);
     }
     mbar_init(BAR(B_SFULL), 1);
-    mbar_init(BAR(B_SFULL + 1), 1);
+    mbar_init(BAR(B_SFREE), kBwdCompute);
     mbar_init(BAR(B_DPFULL), 1);
+    mbar_init(BAR(B_DPFULL + 1), 1);
     mbar_init(BAR(B_DSREADY), kBwdCompute);
     mbar_init(BAR(B_DONE), 1);
     mbar_init(BAR(B_DRAIN), 1);
@@ -756,31 +776,37 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         const int kvrow = it.b * p.Hkv + it.h / p.group;
         for (int st = 0; st < it.n && ok; ++st) {
           const int kt = it.kt_lo + st;
-          const uint32_t slot = lidx % C::NST;
-          if (!wait_bounded(BAR(B_KVEMPTY + slot), ((lidx / C::NST) & 1) ^ 1, abort_flag, tmo)) { ok = false; break; }
-          const uint32_t stage = sbase + C::OFF_RING + slot * 2 * C::TILE_BYTES;
-          mbar_expect_tx(BAR(B_KVFULL + slot), 2 * C::TILE_BYTES);
-          for (int pn = 0; pn < C::NPANEL; ++pn) {
-            tma_load_3d(stage + pn * C::PANEL_BYTES, &tm_k, BAR(B_KVFULL + slot), pn * 64, kt * 128, kvrow, pol_last);
-            tma_load_3d(stage + C::TILE_BYTES + pn * C::PANEL_BYTES, &tm_v, BAR(B_KVFULL + slot), pn * 64, kt * 128,
-                        kvrow, pol_last);
-          }
+          // K and V of step lidx, each into its own ring
+          const uint32_t ks = lidx % NK, vs = lidx % NV;
+          if (!wait_bounded(BAR(B_KEMPTY + ks), ((lidx / NK) & 1) ^ 1, abort_flag, tmo)) { ok = false; break; }
+          mbar_expect_tx(BAR(B_KFULL + ks), C::TILE_BYTES);
+          for (int pn = 0; pn < C::NPANEL; ++pn)
+            tma_load_3d(sbase + C::DQ_OFF_K + ks * C::TILE_BYTES + pn * C::PANEL_BYTES, &tm_k, BAR(B_KFULL + ks),
+                        pn * 64, kt * 128, kvrow, pol_last);
+          if (!wait_bounded(BAR(B_VEMPTY + vs), ((lidx / NV) & 1) ^ 1, abort_flag, tmo)) { ok = false; break; }
+          mbar_expect_tx(BAR(B_VFULL + vs), C::TILE_BYTES);
+          for (int pn = 0; pn < C::NPANEL; ++pn)
+            tma_load_3d(sbase + C::DQ_OFF_V + vs * C::TILE_BYTES + pn * C::PANEL_BYTES, &tm_v, BAR(B_VFULL + vs),
+                        pn * 64, kt * 128, kvrow, pol_last);
           ++lidx;
         }
       }
       if (items > 0) drain_bounded(BAR(B_QFULL), (items - 1) & 1, tmo);
-      for (uint32_t idx = (lidx > C::NST ? lidx - C::NST : 0); idx < lidx; ++idx)
-        drain_bounded(BAR(B_KVFULL + idx % C::NST), (idx / C::NST) & 1, tmo);
+      for (uint32_t idx = (lidx > NK ? lidx - NK : 0); idx < lidx; ++idx)
+        drain_bounded(BAR(B_KFULL + idx % NK), (idx / NK) & 1, tmo);
+      for (uint32_t idx = (lidx > NV ? lidx - NV : 0); idx < lidx; ++idx)
+        drain_bounded(BAR(B_VFULL + idx % NV), (idx / NV) & 1, tmo);
     }
   } else if (warp == kBwdMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t tDP = tbase + C::T_DPQ, tDQ = tbase + C::T_DQ;
-      auto tSb = [&](uint32_t t) -> uint32_t { return tbase + ((t & 1u) ? C::T_SB : C::T_S); };
+      const uint32_t tS = tbase + C::T_S, tDQ = tbase + C::T_DQ;
+      auto tDPb = [&](uint32_t t) -> uint32_t { return tbase + ((t & 1u) ? C::T_DP1 : C::T_DP0); };
       const uint64_t dq_k = make_sdesc_sw128(sbase + C::OFF_A, 16, 1024);
       const uint64_t ddo_k = make_sdesc_sw128(sbase + C::OFF_B, 16, 1024);
-      const uint64_t dring_k = make_sdesc_sw128(sbase + C::OFF_RING, 16, 1024);
-      const uint64_t dring_mn = make_sdesc_sw128(sbase + C::OFF_RING, C::PANEL_BYTES, 1024);
+      const uint64_t dk_k = make_sdesc_sw128(sbase + C::DQ_OFF_K, 16, 1024);                  // K, K-major (S)
+      const uint64_t dk_mn = make_sdesc_sw128(sbase + C::DQ_OFF_K, C::PANEL_BYTES, 1024);     // K, MN-major (dQ)
+      const uint64_t dv_k = make_sdesc_sw128(sbase + C::DQ_OFF_V, 16, 1024);                  // V, K-major (dP)
       auto ss = [&](uint32_t dst, uint64_t a0, uint64_t b0) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -789,9 +815,22 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           mma_f16_ss(dst, a0 + off, b0 + off, C::IDESC_SS, kk > 0);
         }
       };
-      auto soff = [&](uint32_t idx) -> uint32_t { return ((idx % C::NST) * 2 * C::TILE_BYTES) >> 4; };
-      auto kv_ready = [&](uint32_t idx) -> bool {
-        return wait_bounded(BAR(B_KVFULL + idx % C::NST), (idx / C::NST) & 1, abort_flag, tmo);
+      auto koff = [&](uint32_t idx) -> uint32_t { return ((idx % NK) * C::TILE_BYTES) >> 4; };
+      auto voff = [&](uint32_t idx) -> uint32_t { return ((idx % NV) * C::TILE_BYTES) >> 4; };
+      auto k_ready = [&](uint32_t idx) -> bool {
+        return wait_bounded(BAR(B_KFULL + idx % NK), (idx / NK) & 1, abort_flag, tmo);
+      };
+      auto v_ready = [&](uint32_t idx) -> bool {
+        return wait_bounded(BAR(B_VFULL + idx % NV), (idx / NV) & 1, abort_flag, tmo);
+      };
+      // dP of step index idx into dP buffer t & 1; its V slot is free once the MMA is done
+      auto dp_step = [&](uint32_t idx, uint32_t t) -> bool {
+        if (!v_ready(idx)) return false;
+        tc_fence_after();
+        ss(tDPb(t), ddo_k, dv_k + voff(idx));
+        mma_commit(BAR(B_DPFULL + (t & 1)));
+        mma_commit(BAR(B_VEMPTY + idx % NV));
+        return true;
       };
       uint32_t items = 0, cidx = 0, tcount = 0;
       bool ok = true;
@@ -800,39 +839,32 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         if (w >= p.num_items) break;
         const QItem it = make_q_item(p, w);
         if (it.n == 0) continue;
-        if (!wait_bounded(BAR(B_QFULL), items & 1, abort_flag, tmo) || !kv_ready(cidx)) { ok = false; break; }
+        if (!wait_bounded(BAR(B_QFULL), items & 1, abort_flag, tmo) || !k_ready(cidx)) { ok = false; break; }
         tc_fence_after();
-        // S(0) = Q K^T and dP(0) = dO V^T; S(1) ahead into the other buffer
-        ss(tSb(tcount), dq_k, dring_k + soff(cidx));
-        mma_commit(BAR(B_SFULL + (tcount & 1)));
-        ss(tDP, ddo_k, dring_k + soff(cidx) + (C::TILE_BYTES >> 4));
-        mma_commit(BAR(B_DPFULL));
-        if (it.n > 1) {
-          if (!kv_ready(cidx + 1)) { ok = false; break; }
-          tc_fence_after();
-          ss(tSb(tcount + 1), dq_k, dring_k + soff(cidx + 1));
-          mma_commit(BAR(B_SFULL + ((tcount + 1) & 1)));
-        }
+        // S(0) = Q K^T, dP(0) = dO V^T, and dP(1) ahead into the other dP buffer
+        ss(tS, dq_k, dk_k + koff(cidx));
+        mma_commit(BAR(B_SFULL));
+        if (!dp_step(cidx, tcount) || (it.n > 1 && !dp_step(cidx + 1, tcount + 1))) { ok = false; break; }
         for (int st = 0; st < it.n; ++st) {
           const uint32_t idx = cidx + st, t = tcount + st;
-          // dQ += dS K once dS is written (over S of this step)
+          // S of the next step once the compute warps have read this one
+          if (!wait_bounded(BAR(B_SFREE), t & 1, abort_flag, tmo)) { ok = false; break; }
+          if (st + 1 < it.n) {
+            if (!k_ready(idx + 1)) { ok = false; break; }
+            tc_fence_after();
+            ss(tS, dq_k, dk_k + koff(idx + 1));
+            mma_commit(BAR(B_SFULL));
+          }
+          // dQ += dS K once dS is written (over this step's dP); then K of this step is free
           if (!wait_bounded(BAR(B_DSREADY), t & 1, abort_flag, tmo)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_f16_ts(tDQ, tSb(t) + kk * 8, dring_mn + soff(idx) + ((kk * 16 * 128) >> 4), C::IDESC_TS,
+            mma_f16_ts(tDQ, tDPb(t) + kk * 8, dk_mn + koff(idx) + ((kk * 16 * 128) >> 4), C::IDESC_TS,
                        (st > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(BAR(B_KVEMPTY + idx % C::NST));
-          if (st + 1 < it.n) {   // dP of the next step (its K/V stage was waited for above)
-            ss(tDP, ddo_k, dring_k + soff(idx + 1) + (C::TILE_BYTES >> 4));
-            mma_commit(BAR(B_DPFULL));
-          }
-          if (st + 2 < it.n) {   // S two steps ahead, into the buffer dQ has just read
-            if (!kv_ready(idx + 2)) { ok = false; break; }
-            tc_fence_after();
-            ss(tSb(t), dq_k, dring_k + soff(idx + 2));
-            mma_commit(BAR(B_SFULL + (t & 1)));
-          }
+          mma_commit(BAR(B_KEMPTY + idx % NK));
+          // dP two steps ahead, into the buffer dQ has just read
+          if (st + 2 < it.n && !dp_step(idx + 2, t)) { ok = false; break; }
         }
         if (!ok) break;
         mma_commit(BAR(B_QEMPTY));
@@ -849,7 +881,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const int quarter = warp & 3, half = warp >> 2;
     const int rloc = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t tDP = tbase + C::T_DPQ + lane_off;
+    const uint32_t tS = tbase + C::T_S + lane_off;
     const int col0 = 64 * half;                              // this warp's key columns col0 .. col0+63
     uint32_t tcount = 0, items = 0;
     bool ok = true;
@@ -892,9 +924,8 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       for (int st = 0; st < it.n; ++st) {
         const uint32_t t = tcount + st;
         const int kt = it.kt_lo + st;
-        const uint32_t tS = tbase + ((t & 1u) ? C::T_SB : C::T_S) + lane_off;
-        if (!__all_sync(0xffffffffu, wait_bounded(BAR(B_SFULL + (t & 1)), (t >> 1) & 1, abort_flag, tmo) &&
-                                     wait_bounded(BAR(B_DPFULL), t & 1, abort_flag, tmo))) {
+        const uint32_t tDP = tbase + ((t & 1u) ? C::T_DP1 : C::T_DP0) + lane_off;
+        if (!__all_sync(0xffffffffu, wait_bounded(BAR(B_SFULL), t & 1, abort_flag, tmo))) {
           ok = false;
           break;
         }
@@ -913,23 +944,33 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         uint32_t sa[32], sb[32];
         tmem_ld_x32_wait(tS + col0, sa);
         tmem_ld_x32_wait(tS + col0 + 32, sb);
-        // every warp has read its S columns before any dS is written over them
-        if (!compute_sync(BAR(B_SYNC), t & 1, abort_flag, tmo)) { ok = false; break; }
+        // S is in registers: the MMA may compute the next step's S over it
+        tc_fence_before();
+        mbar_arrive(BAR(B_SFREE));
         // P * dt/ds rounded to bf16 first, as in the dK/dV kernel, so that both use the same dS
         uint32_t pk[32], pf[32];
         auto lse_at = [&](int) -> float { return lse2; };
         if (full) p_loop<false, SOFTCAP, ALIBI, 1>(p, sa, sb, vm, slope_l2, rel0, lse_at, pk, pf);
         else p_loop<true, SOFTCAP, ALIBI, 1>(p, sa, sb, vm, slope_l2, rel0, lse_at, pk, pf);
+        if (!__all_sync(0xffffffffu, wait_bounded(BAR(B_DPFULL + (t & 1)), (t >> 1) & 1, abort_flag, tmo))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t da[32], db[32];
+        tmem_ld_x32_wait(tDP + col0, da);
+        tmem_ld_x32_wait(tDP + col0 + 32, db);
+        // every warp has read its dP columns before any dS is written over them
+        if (!compute_sync(BAR(B_SYNC), t & 1, abort_flag, tmo)) { ok = false; break; }
         uint32_t dk[32];
-        uint32_t dq32[32];                                   // 32 columns of dP at a time
 #pragma unroll
         for (int e = 0; e < 64; e += 2) {
-          if ((e & 31) == 0) tmem_ld_x32_wait(tDP + col0 + e, dq32);
           const float2 pp = unpack_bf16x2(pf[e >> 1]);
-          dk[e >> 1] = pack_bf16x2(pp.x * (__uint_as_float(dq32[e & 31]) - dvi),
-                                   pp.y * (__uint_as_float(dq32[(e + 1) & 31]) - dvi));
+          const float x0 = __uint_as_float(e < 32 ? da[e] : db[e - 32]);
+          const float x1 = __uint_as_float(e + 1 < 32 ? da[e + 1] : db[e + 1 - 32]);
+          dk[e >> 1] = pack_bf16x2(pp.x * (x0 - dvi), pp.y * (x1 - dvi));
         }
-        tmem_st_x32_wait<0>(tS + (col0 >> 1), dk);   // dS: key pair (2c, 2c+1) in column c
+        tmem_st_x32_wait<0>(tDP + (col0 >> 1), dk);   // dS: key pair (2c, 2c+1) in column c
         tc_fence_before();
         mbar_arrive(BAR(B_DSREADY));
       }
