@@ -615,6 +615,9 @@ def main():
     ap.add_argument("--heads", type=int, default=0, help="override H (smaller ncu captures)")
     ap.add_argument("--backward", action="store_true",
                     help="with --kernel-only: time attn_bwd (dQ, dK, dV) of the workload instead of the forward")
+    ap.add_argument("--pair", action="store_true",
+                    help="with --kernel-only: time the forward through attn_fwd_pair (2-CTA clusters; "
+                         "BF16 batched workloads with D = 128)")
     ap.add_argument("--tau", type=float, default=None,
                     help="ablation builds only (TILED_ATTENTION_LIB=.../libattn_abl*.so): rescale threshold; "
                          "the line then reports the rescale counters")
@@ -657,6 +660,14 @@ def main():
     case = Case(ta, w, dev, seed=rank)
     stream = torch.cuda.current_stream(dev)
     quant_ms = case.quantize_ms() if w.fp8 else None
+    if args.pair:
+        if not args.kernel_only or args.backward or w.fp8 or w.varlen or w.D != 128:
+            ap.error("--pair needs --kernel-only and a BF16 batched forward workload with D = 128")
+
+        def pair_step():
+            ta.attn_fwd_pair(case.q, case.k, case.v, o=case.o, lse=case.lse, scale=w.scale, mask_kind=w.mask_kind,
+                             window=w.window, softcap=w.softcap, alibi_slopes=case.sl, doc_ids=case.doc)
+        case.step = pair_step
     if args.backward:
         if not args.kernel_only or w.fp8 or w.varlen:
             ap.error("--backward needs --kernel-only and a BF16 batched workload")
@@ -721,6 +732,7 @@ def main():
             line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
                     "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
                     "config": workload_config(w), "kernel_only": True, "backward": args.backward,
+                    "pair": args.pair,
                     "gpu_launches": case.launches_per_step * args.steps}
             if ablation is not None:
                 line["ablation"] = ablation
