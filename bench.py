@@ -629,6 +629,11 @@ def main():
         import dataclasses
         w = dataclasses.replace(w, H=args.heads, note=w.note.replace(f"H{w.H}", f"H{args.heads}"))
 
+    if args.pair and (not args.kernel_only or args.backward or w.fp8 or w.varlen or w.D != 128):
+        ap.error("--pair needs --kernel-only and a BF16 batched forward workload with D = 128")
+    if args.backward and (not args.kernel_only or w.fp8 or w.varlen):
+        ap.error("--backward needs --kernel-only and a BF16 batched workload")
+
     if args.impl == "reference":
         run_reference(args, w)
         return
@@ -661,16 +666,11 @@ def main():
     stream = torch.cuda.current_stream(dev)
     quant_ms = case.quantize_ms() if w.fp8 else None
     if args.pair:
-        if not args.kernel_only or args.backward or w.fp8 or w.varlen or w.D != 128:
-            ap.error("--pair needs --kernel-only and a BF16 batched forward workload with D = 128")
-
         def pair_step():
             ta.attn_fwd_pair(case.q, case.k, case.v, o=case.o, lse=case.lse, scale=w.scale, mask_kind=w.mask_kind,
                              window=w.window, softcap=w.softcap, alibi_slopes=case.sl, doc_ids=case.doc)
         case.step = pair_step
     if args.backward:
-        if not args.kernel_only or w.fp8 or w.varlen:
-            ap.error("--backward needs --kernel-only and a BF16 batched workload")
         case.step()
         g = torch.Generator().manual_seed(1)
         do = torch.randn(case.o.shape, generator=g).to(torch.bfloat16).to(dev)

@@ -51,6 +51,19 @@ def test_reference_arm_prints_one_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0
 
 
+@pytest.mark.parametrize("argv", [["--pair"], ["--pair", "--kernel-only", "--workload", "fp8"],
+                                  ["--pair", "--kernel-only", "--workload", "tiny"],
+                                  ["--pair", "--kernel-only", "--backward"], ["--backward"],
+                                  ["--backward", "--kernel-only", "--workload", "varlen"]])
+def test_mode_flags_rejected_before_any_device_use(argv):
+    """--pair and --backward need --kernel-only and a workload the entry point takes; the
+    error comes from the argument check (exit 2), before any GPU work."""
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py")] + argv, capture_output=True, text=True,
+                       timeout=300)
+    assert r.returncode == 2, (r.returncode, r.stderr[-300:])
+    assert "needs --kernel-only" in r.stderr
+
+
 def test_committed_traffic_files_are_well_formed():
     """Every profiles/traffic_<workload>.json names a known workload, a kernel source hash
     and positive DRAM byte counts whose sum is the per-launch figure."""
