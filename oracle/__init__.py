@@ -15,9 +15,12 @@ Modules
                grouped-query heads and packed variable-length sequences.
 ``attention_bwd``  the gradients dQ, dK, dV of that forward (the chain rule, step by step).
 ``e4m3``       the FP8 e4m3 code book, encoder and per-128-row block quantiser.
+``fp4``        the FP4 e2m1 code book and encoder, the MX (32-element, power-of-two scale)
+               block quantiser, and the Direct-P attention forward that maps scores
+               straight to FP4 codes.
 ``tile_map``   the block-sparse tile classification (EMPTY / PARTIAL / FULL), by brute force.
 
 Every function is pinned by the ``-m "not gpu"`` tests in ``tests/test_oracle_*.py``
 against closed forms, invariants, brute force on tiny inputs and library routines
-(torch's CPU fp64 SDPA, torch's e4m3 cast).  No function is left "parity unpinned".
+(torch's CPU fp64 SDPA, torch's e4m3 cast, ml_dtypes' e2m1 type).  No function is left "parity unpinned".
 """
