@@ -23,13 +23,14 @@ t_ij = scale * log2(e) * (q_i . k_j), with q, k the dequantised inputs.  Keys fo
 of 32 (j // 32), the block scale of P.  For each row and block, E = floor(max t over the
 block's keys) - 2, and each key gets the code
 
-    c = clip(floor(2 (t - E) + KAPPA), 0, 7),   KAPPA = 3 - log2(1.5),
+    c = clip(rint(2 (t - E) + 2), 0, 7)        (rint: nearest integer, ties to even)
 
-i.e. the e2m1 magnitudes read as a logarithmic scale with two codes per octave: c is an
-affine function of the score, floored, with no exponential in between.  KAPPA puts the
-boundaries between codes 2..7 halfway, in log2, between neighbouring magnitudes (1 | 1.5 at
-log2(1.5)/2, 1.5 | 2 at (1 + log2 1.5)/2, and so on each octave).  P~_ij = value(c) * 2^E
-stands for 2^t_ij.  Attention then normalises by what it multiplied:
+i.e. the e2m1 codes read as a logarithmic scale in half octaves (code 2 is 2^0, code 4 is
+2^1, code 6 is 2^2, the odd codes between them): the code is the score itself, rounded to
+the nearest half octave, with no exponential and no rounding of a probability in between.
+P~_ij = value(c) * 2^E, the e2m1 magnitude the tensor core multiplies (the odd codes' 1.5
+sits 0.085 octave above the half-octave point they stand for), represents 2^t_ij.
+Attention then normalises by what it multiplied:
 
     O_i = sum_j P~_ij v_j / sum_j P~_ij,    LSE_i = ln(sum_j P~_ij).
 
@@ -43,7 +44,6 @@ import numpy as np
 
 BLOCK = 32                       # elements per MX scale (Q, K along D; V and P along keys)
 E2M1_MAX = 6.0
-KAPPA = 3.0 - math.log2(1.5)     # Direct-P offset
 LOG2E = 1.0 / math.log(2.0)
 
 
@@ -113,8 +113,8 @@ def mx_dequantize(codes, X, axis: int = -1) -> np.ndarray:
 
 def direct_p_codes(t, E) -> np.ndarray:
     """Direct-P code of scores t (log2 units) against block exponents E (broadcast)."""
-    y2 = 2.0 * (np.asarray(t, dtype=np.float64) - np.asarray(E, dtype=np.float64)) + KAPPA
-    return np.clip(np.floor(y2), 0, 7).astype(np.int64)
+    y2 = 2.0 * (np.asarray(t, dtype=np.float64) - np.asarray(E, dtype=np.float64)) + 2.0
+    return np.clip(np.rint(y2), 0, 7).astype(np.int64)
 
 
 def direct_p_rows(t: np.ndarray):

@@ -91,39 +91,49 @@ def test_mx_padding_of_ragged_axis():
 # ---------------------------------------------------------------- Direct-P
 
 
-def _log_grid():
-    """log2 of the positive magnitudes of codes 1..7, from the code book."""
-    return np.log2(fp4.VALUES[1:8])
+def _half_octave_positions():
+    """Positions, in log2 relative to 2^E, that codes 1..7 stand for, derived from the code
+    book: the even codes 2, 4, 6 at log2 of their magnitudes (1, 2, 4), each odd code halfway
+    between its even neighbours, code 7 half an octave above code 6 and code 1 half an octave
+    below code 2."""
+    L = {c: math.log2(fp4.VALUES[c]) for c in (2, 4, 6)}
+    L[3] = (L[2] + L[4]) / 2
+    L[5] = (L[4] + L[6]) / 2
+    L[7] = L[6] + (L[6] - L[5])
+    L[1] = L[2] - (L[3] - L[2])
+    return np.array([L[c] for c in range(1, 8)])
 
 
-def test_direct_p_codes_at_grid_points():
-    """A score that sits exactly on a magnitude of codes 2..7 (relative to E) gets that code."""
-    lg = _log_grid()
-    for c in range(2, 8):
-        assert fp4.direct_p_codes(lg[c - 1], 0.0) == c
+def test_direct_p_codes_at_even_code_magnitudes():
+    """A score that sits exactly on the magnitude of code 2, 4 or 6 (relative to E) gets it."""
+    for c in (2, 4, 6):
+        assert fp4.direct_p_codes(math.log2(fp4.VALUES[c]), 0.0) == c
 
 
-def test_direct_p_is_nearest_in_log2_for_codes_2_to_7():
-    """From one step below magnitude 1 up to the top of the block's range, the code is the
-    magnitude nearest in log2 (brute force over the code book), saturating at 6."""
-    lg = _log_grid()[1:]                      # codes 2..7
-    y = np.linspace(-0.2, 2.999, 20001)
+def test_direct_p_is_nearest_half_octave_position():
+    """Brute force over the positions derived from the code book: the code is the nearest
+    one; below a quarter octave under code 1's position the code is 0."""
+    pos = _half_octave_positions()
+    y = np.linspace(-3.0, 2.999, 60001)
     got = fp4.direct_p_codes(y, 0.0)
-    d = np.abs(y[:, None] - lg[None, :])
-    ref = 2 + np.argmin(d, axis=1)
+    d = np.abs(y[:, None] - pos[None, :])
+    ref = 1 + np.argmin(d, axis=1)
+    ref = np.where(y < pos[0] - (pos[1] - pos[0]) / 2, 0, ref)
     srt = np.sort(d, axis=1)
-    clear = srt[:, 1] - srt[:, 0] > 1e-9
+    clear = (srt[:, 1] - srt[:, 0] > 1e-9) & (np.abs(y - (pos[0] - 0.25)) > 1e-9)
     assert np.array_equal(got[clear], ref[clear])
 
 
 def test_direct_p_ratio_bound_and_monotone():
+    """For codes 2..7 the multiplied magnitude is within [0.75, 1.5 / 2^0.25] of 2^y (the odd
+    codes' 1.5 and the saturated top code set the ends); the map is monotone."""
     rng = np.random.default_rng(4)
-    y = np.sort(rng.uniform(-0.2075, 3.0, size=100000))
+    y = np.sort(rng.uniform(-0.2499, 3.0, size=100000))
     c = fp4.direct_p_codes(y, 0.0)
-    assert np.all(np.diff(c) >= 0)
+    assert np.all(np.diff(c) >= 0) and c.min() >= 2
     ratio = fp4.VALUES[c] / np.exp2(y)
-    assert np.all(ratio >= 2.0 ** -0.415 - 1e-12)
-    assert np.all(ratio <= 2.0 ** (math.log2(1.5) / 2) + 1e-12)
+    assert np.all(ratio >= 0.75 - 1e-12)
+    assert np.all(ratio <= 1.5 / 2.0 ** 0.25 + 1e-12)
     yy = np.linspace(-20, 3, 5000)
     cc = fp4.direct_p_codes(yy, 0.0)
     assert np.all(np.diff(cc) >= 0) and cc[0] == 0 and cc[-1] == 7
@@ -190,12 +200,11 @@ def test_golden_worked_examples():
 
 
 def _brute_force(q, k, v, scale):
-    """Pure-Python loops.  Code boundaries come from the code book: halfway in log2 between
-    neighbouring magnitudes of codes 2..7, and the same half-octave spacing continued below
-    code 3 (boundaries of codes 2 and 1)."""
+    """Pure-Python loops.  Code boundaries come from the code book: halfway between the
+    half-octave positions of neighbouring codes (positions from the even codes' magnitudes)."""
     mags = [float(fp4.VALUES[c]) for c in range(8)]
-    mid = [(math.log2(mags[c - 1]) + math.log2(mags[c])) / 2 for c in range(3, 8)]   # codes 3..7
-    bounds = [mid[0] - 1.0, mid[0] - 0.5] + mid                                     # codes 1..7
+    pos = [float(x) for x in _half_octave_positions()]                             # codes 1..7
+    bounds = [pos[0] - (pos[1] - pos[0]) / 2] + [(pos[c] + pos[c + 1]) / 2 for c in range(6)]
     Sq, D = len(q), len(q[0])
     Sk = len(k)
     out, lse = [], []
