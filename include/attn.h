@@ -268,6 +268,42 @@ ATTN_API int attn_fwd_fp8(const void* q8, const void* k8, const void* v8,
                  const float* alibi_slopes, const int* doc_ids, void* stream);
 
 /*
+ * attn_quantize_mxfp4 — MXFP4 quantiser for the FP4 forward (page "Hardware-Aware FP4
+ * FlashAttention-4", summary paragraph: the forward runs on the FP4 tensor cores).  Element
+ * format e2m1; one power-of-two scale per 32 consecutive elements of the contraction axis,
+ * stored as the E8M0 byte X + 127 with X = floor(log2 max|x|) - 2 (an all-zero block stores
+ * 0); element = e2m1 round-to-nearest-even, saturating at 6, of x * 2^-X.
+ *   x     device bf16 [B,H,S,D], D = 128 (read)
+ *   transpose = 0 (Q, K): xq bytes [B,H,S,64] (element d in byte d/2, low nibble for even d);
+ *       x_sf bytes [B,H,ceil(S/128),512] (written).
+ *   transpose = 1 (V): xq bytes [B,H,128,Sp/2], Sp = S rounded up to 128 (row d holds the
+ *       keys; keys >= S are zero); x_sf bytes [B,H,Sp/128,512] (written).
+ * Scale atom layout (what the tensor core reads, 128 rows x 4 blocks per 512 bytes): the
+ * scale of row r (0..127 within the atom) and block k (0..3) is byte 16*(r%32) + 4*(r/32) + k.
+ * Rows of the last atom past S get scale byte 0.  Pointers 16-byte aligned.  Returns
+ * ATTN_ERR_INVALID for a bad argument (nothing launched).
+ */
+ATTN_API int attn_quantize_mxfp4(const void* x, void* xq, void* x_sf, int B, int H, int S, int D,
+                                 int transpose, void* stream);
+
+/*
+ * attn_fwd_fp4 — attention forward for non-causal inference on MXFP4 Q, K, V with Direct-P
+ * (page "Hardware-Aware FP4 FlashAttention-4", Direct-P paragraphs: the scores are mapped
+ * straight to the FP4 codes the tensor cores multiply).  Both products run on the FP4 tensor
+ * cores.  P: for each row and block of 32 keys, E = floor(max t) - 2 with t = scale *
+ * log2(e) * s; code = clip(rint(2 (t - E) + 2), 0, 7) (the score rounded to the nearest
+ * half octave above 2^E), block scale 2^E.  O = sum P~ v / sum P~ and LSE = ln(sum P~), P~
+ * the e2m1 magnitudes times the block scales.  No mask (all keys < Sk visible).
+ *   q4 [B,H,Sq,64], k4 [B,H_kv,Sk,64], vt4 [B,H_kv,128,Sp/2] and their scale atoms, as
+ *   attn_quantize_mxfp4 writes them (D = 128); o bf16 [B,H,Sq,128]; lse fp32 [B,H,Sq].
+ * H must be a multiple of H_kv (query head h reads key/value head h / (H/H_kv)).  Device
+ * pointers, 16-byte aligned, caller-owned; nothing is allocated.  Errors as attn_fwd.
+ */
+ATTN_API int attn_fwd_fp4(const void* q4, const void* k4, const void* vt4, const void* q_sf,
+                          const void* k_sf, const void* v_sf, void* o, float* lse, int B, int H,
+                          int H_kv, int Sq, int Sk, float scale, void* stream);
+
+/*
  * attn_get_status — synchronises `stream`, then returns and clears the current device's
  * status word: ATTN_OK, or ATTN_ERR_TIMEOUT if a kernel's bounded wait ran out since the
  * last call (that kernel abandoned its work item and left its outputs undefined),

@@ -72,6 +72,25 @@ def test_bad_arguments_other_entry_points():
     assert lib.attn_fwd_fp8(*fp8) == _lib.ATTN_ERR_INVALID          # missing scales
 
 
+@pytest.mark.parametrize("i,val", [(0, None), (3, None), (5, None), (6, None), (7, None), (2, A + 8),
+                                   (8, 0), (9, 0), (10, 3), (11, 0), (12, -1), (11, (1 << 20) + 1),
+                                   (13, 0.0), (13, float("nan"))])
+def test_fp4_forward_rejects_bad_arguments(i, val):
+    # q4, k4, vt4, q_sf, k_sf, v_sf, o, lse, B, H, H_kv, Sq, Sk, scale
+    args = [A, A, A, A, A, A, A, A, 1, 2, 1, 128, 128, 0.1]
+    args[i] = val
+    assert _lib.load().attn_fwd_fp4(*args, None) == _lib.ATTN_ERR_INVALID
+
+
+@pytest.mark.parametrize("kw", [dict(x=None), dict(D=64), dict(S=0), dict(transpose=2), dict(xq=A + 4),
+                                dict(S=(1 << 20) + 1)])
+def test_mxfp4_quantiser_rejects_bad_arguments(kw):
+    a = dict(x=A, xq=A, sf=A, B=1, H=1, S=128, D=128, transpose=0)
+    a.update(kw)
+    assert _lib.load().attn_quantize_mxfp4(a["x"], a["xq"], a["sf"], a["B"], a["H"], a["S"], a["D"],
+                                           a["transpose"], None) == _lib.ATTN_ERR_INVALID
+
+
 def test_wrapper_raises_on_missing_library(monkeypatch, tmp_path):
     monkeypatch.setattr(_lib, "_lib", None)
     monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "nope.so"))

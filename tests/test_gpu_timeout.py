@@ -58,3 +58,23 @@ def test_pair_kernel_skipped_signal_times_out_and_context_survives():
     assert ta.attn_get_status() == _lib.ATTN_OK
     O, L, E = oracle_eav(q, k, v, 1.0 / 128 ** 0.5, MASK_CAUSAL)
     compare(o, lse, O, L, eav=E)
+
+
+def test_fp4_kernel_skipped_signal_times_out_and_context_survives():
+    """The same hook in the FP4 kernel: query group 1 skips its first P-ready arrival; the
+    MMA issuer's wait runs out, every role unwinds, and the next call is correct."""
+    import tiled_attention_14_b200 as ta
+    from tiled_attention_14_b200 import _lib
+    from tests.test_gpu_fp4 import _check, _quantise_all
+    lib = _lib.load()
+    q, k, v = make_qkv(1, 2, 512, 512, 128, seed=43)
+    q4, qsf, k4, ksf, v4, vsf = _quantise_all(q, k, v)
+    assert ta.attn_get_status() == _lib.ATTN_OK
+    lib.attn_debug_set_fault(1, 200)
+    try:
+        ta.attn_fwd_fp4(q4, qsf, k4, ksf, v4, vsf, 512)
+        assert ta.attn_get_status() == _lib.ATTN_ERR_TIMEOUT
+    finally:
+        lib.attn_debug_set_fault(0, 1000)
+    assert ta.attn_get_status() == _lib.ATTN_OK
+    _check(q, k, v)

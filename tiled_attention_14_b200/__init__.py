@@ -14,6 +14,7 @@ from ._lib import (ATTN_ERR_TIMEOUT, ATTN_OK, MASK_CAUSAL, MASK_DOC, MASK_NONE, 
                    AttnError, check, load)
 
 __all__ = ["attn_fwd", "attn_fwd_pair", "attn_bwd", "attn_fwd_varlen", "attn_fwd_noalloc", "attn_fwd_with_map", "attn_fwd_fp8", "attn_quantize_e4m3",
+           "attn_quantize_mxfp4", "attn_fwd_fp4", "mxfp4_shapes",
            "attn_tile_map_build", "attn_get_status", "attn_shutdown", "tile_map_shape",
            "AttnError", "MASK_NONE", "MASK_CAUSAL", "MASK_WINDOW", "MASK_DOC"]
 
@@ -284,6 +285,75 @@ def attn_fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o=None, lse=None, scale=
                           _ptr(o), _ptr(lse), B, H, Sq, Sk, D, float(scale), int(mask_kind), int(window),
                           float(softcap), _ptr(alibi_slopes), _ptr(doc_ids), _stream(stream))
     check(rc, "attn_fwd_fp8")
+    return o, lse
+
+
+def mxfp4_shapes(B, H, S, transpose=False):
+    """Shapes of (codes, scale atoms) that attn_quantize_mxfp4 writes for a [B,H,S,128] input."""
+    nt = (S + 127) // 128
+    if transpose:
+        return (B, H, 128, nt * 64), (B, H, nt, 512)
+    return (B, H, S, 64), (B, H, nt, 512)
+
+
+def attn_quantize_mxfp4(x, transpose=False, xq=None, x_sf=None, stream=None):
+    """bf16 [B,H,S,128] -> (e2m1 codes uint8, E8M0 scale atoms uint8), MXFP4 (32-element
+    blocks).  transpose=True stores the codes as rows of D holding the keys (the layout V
+    takes in attn_fwd_fp4)."""
+    lib = load()
+    if not isinstance(x, torch.Tensor) or x.dim() != 4 or x.device.type != "cuda":
+        raise ValueError("x: expected a 4-d CUDA tensor [B, H, S, 128]")
+    B, H, S, D = x.shape
+    if D != 128:
+        raise ValueError("attn_quantize_mxfp4 needs D = 128")
+    _need(x, "x", torch.bfloat16, (B, H, S, D), x.device)
+    qshape, sshape = mxfp4_shapes(B, H, S, transpose)
+    if xq is None:
+        xq = torch.empty(qshape, dtype=torch.uint8, device=x.device)
+    else:
+        _need(xq, "xq", torch.uint8, qshape, x.device)
+    if x_sf is None:
+        x_sf = torch.empty(sshape, dtype=torch.uint8, device=x.device)
+    else:
+        _need(x_sf, "x_sf", torch.uint8, sshape, x.device)
+    rc = lib.attn_quantize_mxfp4(_ptr(x), _ptr(xq), _ptr(x_sf), B, H, S, D, 1 if transpose else 0, _stream(stream))
+    check(rc, "attn_quantize_mxfp4")
+    return xq, x_sf
+
+
+def attn_fwd_fp4(q4, q_sf, k4, k_sf, vt4, v_sf, Sk, o=None, lse=None, scale=None, stream=None):
+    """FP4 forward with Direct-P (no mask) on attn_quantize_mxfp4 outputs: q4/q_sf from Q,
+    k4/k_sf from K, vt4/v_sf from V with transpose=True; Sk is the key count.  Grouped heads
+    when K/V have fewer heads than Q.  Returns (o bf16 [B,H,Sq,128], lse fp32 [B,H,Sq])."""
+    lib = load()
+    for name, t in (("q4", q4), ("k4", k4), ("vt4", vt4)):
+        if not isinstance(t, torch.Tensor) or t.dim() != 4 or t.device.type != "cuda":
+            raise ValueError(f"{name}: expected a 4-d CUDA tensor")
+    B, H, Sq, _ = q4.shape
+    Hkv = k4.shape[1]
+    if Hkv <= 0 or H % Hkv != 0:
+        raise ValueError("the query heads must be a multiple of the key/value heads")
+    qs, qsf = mxfp4_shapes(B, H, Sq)
+    ks, ksf = mxfp4_shapes(B, Hkv, Sk)
+    vs, vsf = mxfp4_shapes(B, Hkv, Sk, transpose=True)
+    _need(q4, "q4", torch.uint8, qs, q4.device)
+    _need(q_sf, "q_sf", torch.uint8, qsf, q4.device)
+    _need(k4, "k4", torch.uint8, ks, q4.device)
+    _need(k_sf, "k_sf", torch.uint8, ksf, q4.device)
+    _need(vt4, "vt4", torch.uint8, vs, q4.device)
+    _need(v_sf, "v_sf", torch.uint8, vsf, q4.device)
+    if o is None:
+        o = torch.empty(B, H, Sq, 128, dtype=torch.bfloat16, device=q4.device)
+    else:
+        _need(o, "o", torch.bfloat16, (B, H, Sq, 128), q4.device)
+    if lse is None:
+        lse = torch.empty(B, H, Sq, dtype=torch.float32, device=q4.device)
+    else:
+        _need(lse, "lse", torch.float32, (B, H, Sq), q4.device)
+    scale = 1.0 / math.sqrt(128) if scale is None else scale
+    rc = lib.attn_fwd_fp4(_ptr(q4), _ptr(k4), _ptr(vt4), _ptr(q_sf), _ptr(k_sf), _ptr(v_sf), _ptr(o), _ptr(lse),
+                          B, H, Hkv, Sq, Sk, float(scale), _stream(stream))
+    check(rc, "attn_fwd_fp4")
     return o, lse
 
 

@@ -37,6 +37,8 @@ SIGNATURES = {
     "attn_fwd_with_map": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _F, _P, _P, _P, _P, _P]),
     "attn_quantize_e4m3": (_I, [_P, _P, _P, _I, _I, _I, _I, _P]),
     "attn_fwd_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _F, _P, _P, _P]),
+    "attn_quantize_mxfp4": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P]),
+    "attn_fwd_fp4": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "attn_get_status": (_I, [_P]),
     "attn_strerror": (ctypes.c_char_p, [_I]),
     "attn_shutdown": (None, []),

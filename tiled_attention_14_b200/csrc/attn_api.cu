@@ -18,6 +18,7 @@
 #endif
 #include "attn_bwd_kernel.cuh"
 #include "attn_fwd_kernel.cuh"
+#include "attn_fp4_kernel.cuh"
 #include "attn_fwd_pair_kernel.cuh"
 #include "quant_kernel.cuh"
 #include "tile_map_kernel.cuh"
@@ -436,6 +437,7 @@ int run_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* 
 }
 
 #include "attn_bwd_api.inc"
+#include "attn_fp4_api.inc"
 
 }  // namespace
 
@@ -503,6 +505,18 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const v
              void* stream) {
   return run_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, H, H_kv, Sq, Sk, D, scale, mask_kind, window, softcap,
                  alibi_slopes, doc_ids, static_cast<cudaStream_t>(stream));
+}
+
+int attn_fwd_fp4(const void* q4, const void* k4, const void* vt4, const void* q_sf, const void* k_sf,
+                 const void* v_sf, void* o, float* lse, int B, int H, int H_kv, int Sq, int Sk, float scale,
+                 void* stream) {
+  return run_fwd_fp4(q4, k4, vt4, q_sf, k_sf, v_sf, o, lse, B, H, H_kv, Sq, Sk, scale,
+                     static_cast<cudaStream_t>(stream));
+}
+
+int attn_quantize_mxfp4(const void* x, void* xq, void* x_sf, int B, int H, int S, int D, int transpose,
+                        void* stream) {
+  return run_quant_mxfp4(x, xq, x_sf, B, H, S, D, transpose, static_cast<cudaStream_t>(stream));
 }
 
 int attn_tile_map_build(int* counts, uint32_t* entries, int B, int Sq, int Sk, int mask_kind, int window,
