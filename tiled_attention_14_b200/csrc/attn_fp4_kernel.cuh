@@ -11,7 +11,8 @@
 //     products are K-major, which FP4 operands require.
 //   P (Direct-P): per row and block of 32 keys, E = floor(max t) - 2 with t the score in log2
 //     units; each key's code is the score rounded to the nearest half octave above 2^E,
-//     c = clip(rint(2 (t - E) + 2), 0, 7) — one FMA into a rounding constant, no exponential.
+//     c = clip(rint(2 (t - E) + 2), 0, 7) — two FMAs (one saturating, one rounding down into a
+//     constant whose last bits then hold the code), no exponential.
 //     The block scale 2^(E - m) (m the row's running reference, an integer) is P's E8M0 scale.
 //   O = sum P~ V / sum P~, LSE = ln(sum P~), with P~ the magnitudes the tensor core multiplied.
 //
@@ -117,6 +118,17 @@ __device__ __forceinline__ void tma_load_box(uint32_t dst, const void* map, uint
       " [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(dst),
       "l"(map), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "l"(policy)
       : "memory");
+}
+
+// Two fp32 FMAs in one instruction, rounded toward minus infinity.
+__device__ __forceinline__ float2 ffma2_rm(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rm.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
 }
 
 // 2^e as a float for integer e (0 below the normal range).
@@ -259,10 +271,12 @@ struct Cfg {
   static constexpr int OFF_PSF = OFF_P + 4 * P_TILE;       // P scale atoms [g][buf]
   static constexpr int OFF_BAR = OFF_PSF + 4 * SF;
   // barriers: QFULL 2, QEMPTY 2, KVFULL NS, KVEMPTY NS, SFULL 2, SFREE 2, PFULL 4, PFREE 4,
-  // PVDONE 2, DRAIN 1
+  // DRAIN 1.  "P V of tile k of group g is complete" is read from PFREE[g][k & 1]: the
+  // softmax waited for that barrier's previous phase before writing P of tile k, so the
+  // parity it waits for next is never ambiguous.
   static constexpr int B_QFULL = 0, B_QEMPTY = 2, B_KVFULL = 4, B_KVEMPTY = 4 + NS, B_SFULL = 4 + 2 * NS,
                        B_SFREE = B_SFULL + 2, B_PFULL = B_SFREE + 2, B_PFREE = B_PFULL + 4,
-                       B_PVDONE = B_PFREE + 4, B_DRAIN = B_PVDONE + 2, NBAR = B_DRAIN + 1;
+                       B_DRAIN = B_PFREE + 4, NBAR = B_DRAIN + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
@@ -306,7 +320,6 @@ attn_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       mbar_init(BAR(C::B_QEMPTY + g), 1);
       mbar_init(BAR(C::B_SFULL + g), 1);
       mbar_init(BAR(C::B_SFREE + g), 128);
-      mbar_init(BAR(C::B_PVDONE + g), 1);
       for (int b = 0; b < 2; ++b) {
         mbar_init(BAR(C::B_PFULL + 2 * g + b), 128);
         mbar_init(BAR(C::B_PFREE + 2 * g + b), 1);
@@ -440,7 +453,6 @@ attn_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
               mma_mxf4(tO[g], a, b, idesc_mxf4(128, 128, 0, 2 * (jp & 1)), tsfp, tbase + C::T_SFV + 4 * slot,
                        jp > 0 ? 1u : 0u);
               mma_commit(BAR(C::B_PFREE + 2 * g + buf));
-              mma_commit(BAR(C::B_PVDONE + g));
             }
             if (!ok) break;
             if (jp & 1) mma_commit(BAR(C::B_KVEMPTY + slot));
@@ -493,16 +505,13 @@ attn_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         float bm[2];
 #pragma unroll
         for (int blk = 0; blk < 2; ++blk) {
-          float a0 = kNegInfF, a1 = kNegInfF, a2 = kNegInfF;
+          float a[4] = {kNegInfF, kNegInfF, kNegInfF, kNegInfF};
 #pragma unroll
-          for (int c = 0; c < 30; c += 3) {
-            a0 = fmaxf(a0, __uint_as_float(s[32 * blk + c]));
-            a1 = fmaxf(a1, __uint_as_float(s[32 * blk + c + 1]));
-            a2 = fmaxf(a2, __uint_as_float(s[32 * blk + c + 2]));
-          }
-          a0 = fmaxf(a0, __uint_as_float(s[32 * blk + 30]));
-          a1 = fmaxf(a1, __uint_as_float(s[32 * blk + 31]));
-          bm[blk] = fmaxf(a0, fmaxf(a1, a2));
+          for (int c = 0; c < 32; c += 8)
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              a[u] = fmax3f(a[u], __uint_as_float(s[32 * blk + c + 2 * u]), __uint_as_float(s[32 * blk + c + 2 * u + 1]));
+          bm[blk] = fmax3f(a[0], a[1], fmaxf(a[2], a[3]));
         }
         // block exponents E = floor(max t) - 2 (t = s * c2 / 2), the row reference m
         float E[2];
@@ -523,39 +532,39 @@ attn_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           }
           m = mt;
         }
-        // codes: r = s * c2 + (magic + 2 - 2E) rounds to magic + rint(2 (t - E) + 2)
+        // codes: with y2 = 2 (t - E) + 2, z = sat((y2 + 1/2) / 8) (one FMA with saturation) and
+        // code = floor((8 - 2^-21) z), which is rint(y2) clipped to [0, 7] away from exact ties;
+        // the floor is a round-down FMA into 1.5 * 2^23, whose last bits then hold the code.
         uint32_t pw[8];
         uint32_t sfb = 0;
-        int psum[2];
+        const float a8 = 0.125f * c2;
+        const float2 k8 = make_float2(7.99999952f, 7.99999952f), mg = make_float2(C::kMagic, C::kMagic);
 #pragma unroll
         for (int blk = 0; blk < 2; ++blk) {
           const int e = live[blk] ? static_cast<int>(E[blk] - m) : -1000;   // scale exponent
           const bool use = e >= -127;
-          const float K = use ? (C::kMagic + (2.f - 2.f * E[blk])) : kNegInfF;
+          const float b8 = use ? (2.5f - 2.f * E[blk]) * 0.125f : kNegInfF;
           sfb |= static_cast<uint32_t>(use ? e + 127 : 0) << (8 * blk);
-          uint32_t sum = 0u;
+          uint32_t acc = 0u;   // per-byte sums of twice the magnitudes (at most 96 per byte)
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             uint32_t byte[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
               const int c = 32 * blk + 8 * q + 2 * u;
-              float r0 = fmaf(__uint_as_float(s[c]), c2, K);
-              float r1 = fmaf(__uint_as_float(s[c + 1]), c2, K);
-              r0 = fminf(fmaxf(r0, C::kMagic), C::kMagic + 7.f);
-              r1 = fminf(fmaxf(r1, C::kMagic), C::kMagic + 7.f);
+              const float z0 = __saturatef(fmaf(__uint_as_float(s[c]), a8, b8));
+              const float z1 = __saturatef(fmaf(__uint_as_float(s[c + 1]), a8, b8));
+              const float2 r = ffma2_rm(make_float2(z0, z1), k8, mg);
               // low byte: code1 << 4 | code0 (the constant's low byte is zero)
-              byte[u] = (__float_as_uint(r1) << 4) + __float_as_uint(r0);
+              byte[u] = (__float_as_uint(r.y) << 4) + __float_as_uint(r.x);
             }
             const uint32_t wv = __byte_perm(__byte_perm(byte[0], byte[1], 0x0040), __byte_perm(byte[2], byte[3], 0x0040),
                                             0x5410);
             pw[4 * blk + q] = wv;
-            // twice the magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6} of the 8 codes, summed
-            sum = __dp4a(__byte_perm(0x03020100u, 0x0C080604u, wv), 0x01010101u, sum);
-            sum = __dp4a(__byte_perm(0x03020100u, 0x0C080604u, wv >> 16), 0x01010101u, sum);
+            // twice the magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6} of the 8 codes, byte by byte
+            acc += __byte_perm(0x03020100u, 0x0C080604u, wv) + __byte_perm(0x03020100u, 0x0C080604u, wv >> 16);
           }
-          psum[blk] = use ? static_cast<int>(sum) : 0;
-          if (use) l = fmaf(static_cast<float>(psum[blk]), exp2i(e - 1), l);
+          if (use) l = fmaf(static_cast<float>(__dp4a(acc, 0x01010101u, 0u)), exp2i(e - 1), l);
         }
         // P and its scales to shared memory (buffer buf is free once PV of tile t-2 is done)
         if (t >= 2 && !__all_sync(0xffffffffu, wait_bounded(BAR(C::B_PFREE + 2 * g + buf), ((t >> 1) - 1) & 1,
@@ -571,7 +580,8 @@ attn_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         fence_proxy_async_smem();
         // rescale O when the reference moved (PV of tile t-1 has completed first)
         if (__any_sync(0xffffffffu, rescale)) {
-          if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_PVDONE + g), (t - 1) & 1, abort_flag, tmo))) {
+          if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_PFREE + 2 * g + ((t - 1) & 1)), ((t - 1) >> 1) & 1,
+                                                    abort_flag, tmo))) {
             ok = false;
             break;
           }
@@ -593,7 +603,9 @@ attn_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         break;
       }
       // ---- epilogue: O / l -> bf16, LSE
-      if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_PVDONE + g), (tc + n_sub - 1) & 1, abort_flag, tmo))) {
+      const uint32_t last = tc + n_sub - 1;
+      if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_PFREE + 2 * g + (last & 1)), (last >> 1) & 1, abort_flag,
+                                                tmo))) {
         ok = false;
         break;
       }
