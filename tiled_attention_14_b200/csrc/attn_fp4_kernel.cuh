@@ -268,8 +268,8 @@ struct Cfg {
   static constexpr int STAGE = 17 * 1024;
   static constexpr int OFF_P = OFF_KV + NS * STAGE;        // P[g][buf]: 128 rows x 32 bytes
   static constexpr int P_TILE = 128 * 32;
-  static constexpr int OFF_PSF = OFF_P + 4 * P_TILE;       // P scale atoms [g][buf]
-  static constexpr int OFF_BAR = OFF_PSF + 4 * SF;
+  static constexpr int OFF_PSF = OFF_P + 4 * P_TILE;       // P scale atoms [buf] (both groups)
+  static constexpr int OFF_BAR = OFF_PSF + 2 * SF;
   // barriers: QFULL 2, QEMPTY 2, KVFULL NS, KVEMPTY NS, SFULL 2, SFREE 2, PFULL 4, PFREE 4,
   // DRAIN 1.  "P V of tile k of group g is complete" is read from PFREE[g][k & 1]: the
   // softmax waited for that barrier's previous phase before writing P of tile k, so the
@@ -443,14 +443,20 @@ attn_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const uint32_t tp = tc + jp, buf = tp & 1;
             const uint32_t stage = cidx + (jp >> 1), slot = stage % C::NS;
             const uint32_t st = sbase + C::OFF_KV + slot * C::STAGE;
+            // both groups' P scales share one atom (group g in bytes 2g, 2g + 1 of each row):
+            // one copy to tensor memory serves both products
+            if (!wait_bounded(BAR(C::B_PFULL + buf), (tp >> 1) & 1, abort_flag, tmo) ||
+                !wait_bounded(BAR(C::B_PFULL + 2 + buf), (tp >> 1) & 1, abort_flag, tmo)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t tsfp = tbase + C::T_SFP + 4 * buf;
+            tmem_cp_sf(tsfp, sfdesc(sbase + C::OFF_PSF + buf * C::SF));
             for (int g = 0; g < 2; ++g) {
-              if (!wait_bounded(BAR(C::B_PFULL + 2 * g + buf), (tp >> 1) & 1, abort_flag, tmo)) { ok = false; break; }
-              tc_fence_after();
-              const uint32_t tsfp = tbase + C::T_SFP + 4 * (2 * g + buf);
-              tmem_cp_sf(tsfp, sfdesc(sbase + C::OFF_PSF + (2 * g + buf) * C::SF));
               const uint64_t a = sdesc(sbase + C::OFF_P + (2 * g + buf) * C::P_TILE, 16, 256, kLayoutSw32);
               const uint64_t b = sdesc(st + C::ST_V + 32 * (jp & 1), 16, 512, kLayoutSw64);
-              mma_mxf4(tO[g], a, b, idesc_mxf4(128, 128, 0, 2 * (jp & 1)), tsfp, tbase + C::T_SFV + 4 * slot,
+              mma_mxf4(tO[g], a, b, idesc_mxf4(128, 128, 2 * g, 2 * (jp & 1)), tsfp, tbase + C::T_SFV + 4 * slot,
                        jp > 0 ? 1u : 0u);
               mma_commit(BAR(C::B_PFREE + 2 * g + buf));
             }
@@ -478,7 +484,7 @@ attn_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // P row (32 bytes) of this thread in the 32-byte swizzle: chunk c at c ^ bit 2 of the row
     const uint32_t prow_off = (rloc >> 3) * 256 + (rloc & 7) * 32;
     const uint32_t psw = (rloc >> 2) & 1;
-    const uint32_t psf_off = sf_offset(rloc, 0);
+    const uint32_t psf_off = sf_offset(rloc, 2 * g);
     uint32_t tc = 0;
     bool ok = true;
     for (int w = cta; ok && w < p.num_items; w += G) {
@@ -575,7 +581,7 @@ attn_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         uint8_t* prow = sptr + C::OFF_P + (2 * g + buf) * C::P_TILE + prow_off;
         *reinterpret_cast<uint4*>(prow + (psw << 4)) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
         *reinterpret_cast<uint4*>(prow + ((psw ^ 1u) << 4)) = make_uint4(pw[4], pw[5], pw[6], pw[7]);
-        *reinterpret_cast<uint16_t*>(sptr + C::OFF_PSF + (2 * g + buf) * C::SF + psf_off) =
+        *reinterpret_cast<uint16_t*>(sptr + C::OFF_PSF + buf * C::SF + psf_off) =
             static_cast<uint16_t>(sfb);
         fence_proxy_async_smem();
         // rescale O when the reference moved (PV of tile t-1 has completed first)
