@@ -41,6 +41,7 @@ class Workload:
     alibi: bool = False
     doc: bool = False
     fp8: bool = False
+    fp4: bool = False        # MXFP4 Q/K/V from the bf16 inputs, Direct-P forward (non-causal)
     note: str = ""
     Hkv: int = 0             # key/value heads (0: same as H)
     varlen: bool = False     # packed sequences with the document lengths of doc_lengths()
@@ -69,6 +70,8 @@ WORKLOADS = {
     "doc": Workload("doc", 2, 16, 8192, 8192, 128, MASK_DOC, doc=True,
                     note="B2 H16 S8192 D128 document mask, lengths U[256,2048]"),
     "long": Workload("long", 1, 32, 32768, 32768, 128, note="B1 H32 S32768 D128 non-causal"),
+    "fp4_long": Workload("fp4_long", 1, 32, 32768, 32768, 128, fp4=True,
+                         note="B1 H32 S32768 D128 non-causal, MXFP4 Q/K/V, Direct-P"),
     "fp8": Workload("fp8", 2, 16, 16384, 16384, 128, fp8=True,
                     note="B2 H16 S16384 D128 FP8 e4m3, non-causal"),
     "fp8_causal": Workload("fp8_causal", 2, 16, 16384, 16384, 128, MASK_CAUSAL, fp8=True,

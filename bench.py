@@ -130,7 +130,18 @@ def measured_peaks():
     else:
         out.update(fp8=out["bf16"] * 2.0, fp8_sustained=(out["bf16_sustained"] or 0.0) * 2.0,
                    fp8_source="bf16 x 2 (nominal dense fp8/bf16 ratio)")
+    # no FP4 GEMM is measured: the FP8 figure times the nominal dense FP4/FP8 ratio (9 / 4.5)
+    out.update(fp4=out["fp8"] * 2.0, fp4_sustained=(out["fp8_sustained"] or 0.0) * 2.0,
+               fp4_source=out["fp8_source"] + " x 2 (nominal dense fp4/fp8 ratio)")
     return out
+
+
+def peak_key(w) -> str:
+    return "fp4" if w.fp4 else ("fp8" if w.fp8 else "bf16")
+
+
+def dtype_of(w) -> str:
+    return "e2m1" if w.fp4 else ("e4m3" if w.fp8 else "bf16")
 
 
 class ClockSampler:
@@ -185,9 +196,10 @@ class ClockSampler:
                 "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
-# The sources that make up the forward attention kernel and its launch (the backward,
-# quantiser and tile-map sources do not change it).
-FWD_SOURCES = ("attn_fwd_kernel.cuh", "ptx.cuh", "tmem_moves.cuh", "attn_api.cu")
+# The sources that make up the forward attention kernels (BF16/FP8 and FP4) and their launch
+# (the backward, quantiser and tile-map sources do not change them).
+FWD_SOURCES = ("attn_fwd_kernel.cuh", "ptx.cuh", "tmem_moves.cuh", "attn_api.cu", "attn_fp4_kernel.cuh",
+               "attn_fp4_api.inc")
 
 
 def kernel_source_hash() -> str:
@@ -211,10 +223,45 @@ def profiled_traffic(workload: str):
 
 
 # ----------------------------------------------------------------------------- CPU oracle leg
+_FP4_INPUTS = {}
+
+
+def oracle_sample_fp4(w, budget_s: float, seed: int = 0):
+    """The FP4 oracle on evenly spaced query rows of one (b, h) head: the oracle's MXFP4
+    quantisation of that head's Q, K, V (done once, not timed), then its Direct-P attention
+    in fp64 (timed).  Returns (algorithmic FLOPs done, seconds, description)."""
+    from oracle import fp4
+    key = (w.name, w.Sq, w.Sk, seed)
+    if key not in _FP4_INPUTS:
+        q, k, v = (t.float().numpy() for t in make_qkv(1, 1, w.Sq, w.Sk, w.D, seed=seed))
+
+        def deq(x):
+            c, X = fp4.mx_quantize(x, axis=-1)
+            return fp4.mx_dequantize(c, X, axis=-1)[..., :x.shape[-1]]
+        vh = np.swapaxes(deq(np.swapaxes(v, -1, -2)), -1, -2)
+        _FP4_INPUTS.clear()
+        _FP4_INPUTS[key] = (deq(q), deq(k), vh)
+    qh, kh, vh = _FP4_INPUTS[key]
+    probe = np.arange(min(w.Sq, 64))
+    t0 = time.perf_counter()
+    fp4.attention_fp4_fwd(qh, kh, vh, w.scale, rows=probe)
+    t_probe = time.perf_counter() - t0
+    n = max(len(probe), min(w.Sq, int(len(probe) * budget_s / max(t_probe, 1e-6))))
+    rows = np.linspace(0, w.Sq - 1, num=n).astype(np.int64)
+    t0 = time.perf_counter()
+    fp4.attention_fp4_fwd(qh, kh, vh, w.scale, rows=rows)
+    dt = time.perf_counter() - t0
+    return 4.0 * w.D * w.Sk * len(rows), dt, (f"{len(rows)} of {w.Sq} query rows (evenly spaced) of one (b,h) "
+                                              f"head of the {w.note} workload (Direct-P oracle on the oracle's "
+                                              f"MXFP4 inputs; quantisation not timed)")
+
+
 def oracle_sample(w, budget_s: float, seed: int = 0):
     """Times the fp64 oracle on the workload until about budget_s of CPU work is done:
     whole (b, h) heads while one head fits the budget, else an evenly spaced subset of one
     head's query rows.  Returns (algorithmic FLOPs done, seconds, description)."""
+    if w.fp4:
+        return oracle_sample_fp4(w, budget_s, seed)
     from oracle.attention import attention_fwd, visible_mask
     q, k, v = make_qkv(1, 1, w.Sq, w.Sk, w.D, seed=seed)
     sl = alibi_slopes(w.H)[:1].numpy() if w.alibi else None
@@ -299,7 +346,8 @@ def workload_config(w):
             "mask": {"causal": bool(w.mask_kind & MASK_CAUSAL), "window": w.window,
                      "alibi": w.alibi, "softcap": w.softcap, "document": w.doc},
             "flops": "exact: 4*D per visible (i,j) pair",
-            "l2": f"inputs larger than L2 ({(3 * w.B * w.H * w.Sk * w.D * 2) / 1e6:.0f} MB of Q/K/V + "
+            "l2": f"inputs larger than L2 ({(compulsory_bytes(w) - w.B * w.H * w.Sq * (w.D * 2 + 4)) / 1e6:.0f} MB "
+                  f"of {'MXFP4 ' if w.fp4 else ''}Q/K/V{' and scales' if (w.fp4 or w.fp8) else ''} + "
                   f"{w.B * w.H * w.Sq * w.D * 2 / 1e6:.0f} MB of O vs 126 MB L2); no flush"}
 
 
@@ -340,11 +388,26 @@ class Case:
         if w.fp8:
             # e4m3 operands with per-128-row scales, quantised once (the quantiser is timed alone)
             self.q8 = [ta.attn_quantize_e4m3(t) for t in (self.q, self.k, self.v)]
+        if w.fp4:
+            # MXFP4 operands (V transposed), quantised once (the quantiser is timed alone)
+            self.q4 = self.quantize_fp4(self.q, self.k, self.v)
+
+    def quantize_fp4(self, q, k, v, out=None):
+        ta = self.ta
+        if out is None:
+            return [ta.attn_quantize_mxfp4(q), ta.attn_quantize_mxfp4(k), ta.attn_quantize_mxfp4(v, transpose=True)]
+        for t, tr, (xq, xs) in zip((q, k, v), (False, False, True), out):
+            ta.attn_quantize_mxfp4(t, transpose=tr, xq=xq, x_sf=xs, stream=self.stream)
+        return out
 
     def run(self, q, k, v, quantize=False):
         """The public call a user makes for this workload, on the given inputs."""
         w, ta = self.w, self.ta
-        if w.fp8:
+        if w.fp4:
+            a4 = self.quantize_fp4(q, k, v, out=self.q4) if quantize else self.q4
+            (q4, qs), (k4, ks), (v4, vs) = a4
+            ta.attn_fwd_fp4(q4, qs, k4, ks, v4, vs, w.Sk, o=self.o, lse=self.lse, scale=w.scale)
+        elif w.fp8:
             if quantize:
                 a8 = [ta.attn_quantize_e4m3(t) for t in (q, k, v)]
             else:
@@ -368,6 +431,9 @@ class Case:
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(self.stream)
         for _ in range(reps):
+            if self.w.fp4:
+                self.quantize_fp4(self.q, self.k, self.v, out=self.q4)
+                continue
             for t, (t8, ts) in zip((self.q, self.k, self.v), self.q8):
                 ta.attn_quantize_e4m3(t, t8, ts, stream=self.stream)
         e1.record(self.stream)
@@ -459,6 +525,12 @@ def time_steps(step, n, dev, flush=None):
 
 def compulsory_bytes(w) -> int:
     """Bytes each launch must move at least: Q, K, V read once, O and LSE written once."""
+    if w.fp4:
+        # e2m1 codes (V padded to 128 keys) and their 512-byte scale atoms per 128 rows or keys
+        nq, nk = (w.Sq + 127) // 128, (w.Sk + 127) // 128
+        qkv = w.B * (w.H * w.Sq * 64 + 2 * w.kv_heads * nk * 128 * 64)
+        scales = w.B * (w.H * nq + 2 * w.kv_heads * nk) * 512
+        return qkv + scales + w.B * w.H * w.Sq * (w.D * 2 + 4)
     eb = 1 if w.fp8 else 2
     qkv = w.B * (w.H * w.Sq + 2 * w.kv_heads * w.Sk) * w.D * eb
     scales = 3 * w.B * w.H * ((w.Sk + 127) // 128) * 4 if w.fp8 else 0
@@ -483,18 +555,20 @@ def per_config_record(ta, name, dev, peaks, min_ms=60.0, min_launches=10):
         raise SystemExit(f"kernel status error in workload {name}")
     flops = algorithmic_flops(w)
     tflops = flops / (mean_ms * 1e-3) / 1e12
-    peak = peaks["fp8"] if w.fp8 else peaks["bf16"]
+    peak = peaks[peak_key(w)]
     gbs = compulsory_bytes(w) / (mean_ms * 1e-3) / 1e9
     rec = {"workload": w.note, "steps": n, "timing": how, "ms": mean_ms,
            "tflops_exact": tflops, "peak_tflops": peak, "frac": tflops / peak,
-           "dtype": "e4m3" if w.fp8 else "bf16", "compulsory_bytes": compulsory_bytes(w),
+           "dtype": dtype_of(w), "compulsory_bytes": compulsory_bytes(w),
            "gbs_compulsory": gbs, "hbm_frac": gbs / peaks["hbm"],
            "l2": "flushed before every launch" if flush is not None else "inputs larger than L2",
            "traffic": profiled_traffic(name)}
     if w.doc:
         rec["tile_map_ms"] = case.tile_map_ms()
         rec["attention_ms"] = mean_ms - rec["tile_map_ms"]
-    if w.fp8:
+    if w.fp4:
+        rec["peak_source"] = peaks["fp4_source"]
+    if w.fp8 or w.fp4:
         rec["quantize_ms_per_tensor_set"] = case.quantize_ms()
     del case, flush
     torch.cuda.empty_cache()
@@ -559,7 +633,7 @@ def sustained_record(case, dev, peaks, local, seconds=1.5):
     n = reps * per_graph
     del g
     tflops = algorithmic_flops(case.w) * n / (ms * 1e-3) / 1e12
-    peak = peaks["fp8_sustained"] if case.w.fp8 else peaks["bf16_sustained"]
+    peak = peaks[peak_key(case.w) + "_sustained"]
     return {"launches": n, "ms_total": ms, "tflops_exact": tflops, "peak_tflops": peak,
             "frac": tflops / peak if peak else None,
             "peak_source": "sustained GEMM peak (back-to-back loop under the power cap)",
@@ -629,9 +703,9 @@ def main():
         import dataclasses
         w = dataclasses.replace(w, H=args.heads, note=w.note.replace(f"H{w.H}", f"H{args.heads}"))
 
-    if args.pair and (not args.kernel_only or args.backward or w.fp8 or w.varlen or w.D != 128):
+    if args.pair and (not args.kernel_only or args.backward or w.fp8 or w.fp4 or w.varlen or w.D != 128):
         ap.error("--pair needs --kernel-only and a BF16 batched forward workload with D = 128")
-    if args.backward and (not args.kernel_only or w.fp8 or w.varlen):
+    if args.backward and (not args.kernel_only or w.fp8 or w.fp4 or w.varlen):
         ap.error("--backward needs --kernel-only and a BF16 batched workload")
 
     if args.impl == "reference":
@@ -664,7 +738,7 @@ def main():
                     "lib": os.path.basename(os.environ.get("TILED_ATTENTION_LIB", ""))}
     case = Case(ta, w, dev, seed=rank)
     stream = torch.cuda.current_stream(dev)
-    quant_ms = case.quantize_ms() if w.fp8 else None
+    quant_ms = case.quantize_ms() if (w.fp8 or w.fp4) else None
     if args.pair:
         def pair_step():
             ta.attn_fwd_pair(case.q, case.k, case.v, o=case.o, lse=case.lse, scale=w.scale, mask_kind=w.mask_kind,
@@ -780,20 +854,21 @@ def main():
         # the attention kernel is the dominant launch (one launch per step for analytic masks)
         launch_ms = total_ms / args.steps
         achieved = flops / (launch_ms * 1e-3) / 1e12
-        peak = peaks["fp8"] if w.fp8 else peaks["bf16"]
+        peak = peaks[peak_key(w)]
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "e4m3" if w.fp8 else "bf16",
+            "dtype": dtype_of(w),
             "data": "synthetic", "config": {**workload_config(w), "parallelism": f"replicas x{world}"},
             "tflops_tile_count": weak_scaling_value(tile_count_flops(w), args.steps, world, total_ms),
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": profiled_traffic(args.workload),
-                         "peak_source": (peaks["fp8_source"] if w.fp8 else
+                         "peak_source": (peaks["fp4_source"] if w.fp4 else peaks["fp8_source"] if w.fp8 else
                                          f"bf16_tflops of {peaks['source']} peaks (burst)")
                                         + f"; bf16 sustained {peaks['bf16_sustained']}",
-                         "kernel": "attn_fwd_kernel", "algorithmic_flops_per_launch": flops},
+                         "kernel": "attn_fp4_kernel" if w.fp4 else "attn_fwd_kernel",
+                         "algorithmic_flops_per_launch": flops},
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "clocks": clocks.summary(),
