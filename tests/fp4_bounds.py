@@ -75,7 +75,7 @@ def expected_transposed(v: np.ndarray):
 def dequantised(q, k, v):
     """fp64 Q^, K^, V^ [B, H, S, 128] from the oracle quantiser."""
     out = []
-    for x in (q, k, v):
+    for x in (q, k):
         c, X = fp4.mx_quantize(np.asarray(x, dtype=np.float32), axis=-1)
         out.append(fp4.mx_dequantize(c, X, axis=-1)[..., :x.shape[-1]])
     # V is quantised along the keys (its contraction axis), not along D

@@ -47,3 +47,12 @@ def test_backward_cases(debug_library):
     from tests import test_gpu_bwd as b
     b._run(1, 2, 2, 300, 300, 128, MASK_CAUSAL, seed=9)
     b._run(2, 4, 1, 260, 260, 64, MASK_NONE, softcap=20.0, alibi=True, seed=10)
+
+
+def test_fp4_cases(debug_library):
+    # the FP4 kernel's TMA boxes, bulk scale copies, scale-factor copies to tensor memory and
+    # TMEM moves, and the MXFP4 quantisers, all checked
+    from tests import test_gpu_fp4 as f
+    from attn_workloads import make_qkv
+    f._check(*make_qkv(1, 2, 300, 333, 128, seed=11))
+    f._check(*make_qkv(1, 4, 256, 200, 128, seed=12, Hkv=2))

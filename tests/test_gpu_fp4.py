@@ -100,6 +100,12 @@ def test_fp4_forward_grouped_heads():
     _check(q, k, v)
 
 
+def test_fp4_forward_multi_query_unequal_lengths():
+    """One K/V head for four query heads, more keys than queries (no mask: every key visible)."""
+    q, k, v = make_qkv(2, 4, 300, 700, 128, seed=14, Hkv=1)
+    _check(q, k, v)
+
+
 @pytest.mark.parametrize("mul", [4.0, 0.05])
 def test_fp4_forward_peaked_and_flat_rows(mul):
     """Q x 4 moves the row maximum by many octaves across key tiles (the rescale path);

@@ -1,5 +1,5 @@
 """GPU parity at the longest sequence the C-ABI accepts (Sq = Sk = ATTN_MAX_SEQ = 2^20, one
-head, D = 128), against the fp64 oracle.
+head, D = 128), against the fp64 oracle (the FP4 forward against the FP4 oracle).
 
 Forward: sampled query rows, each exact given the full K and V (first rows, both sides of
 a 256-row block boundary, the middle, the last rows and random ones), with the BF16 gate.
@@ -95,3 +95,12 @@ def test_backward_at_the_maximum_length_causal():
             assert np.all(np.isfinite(gv)), name
             excess = float((np.abs(gv - r) - bd).max())
             assert excess <= 0.0, f"{name}: max|err| {np.abs(gv - r).max():.3e} exceeds the bound by {excess:.3e}"
+
+
+def test_fp4_forward_at_the_maximum_length():
+    """The FP4 Direct-P forward at 2^20 queries and keys, sampled rows, against the FP4 oracle
+    on its own MXFP4 quantisation of the same inputs."""
+    from tests.test_gpu_fp4 import _check
+    q, k, v = _inputs(seed=74)
+    rows = sample_rows(S_MAX, 4, seed=5, extra=[0, 1, S_MAX // 2, S_MAX - 1])
+    _check(q, k, v, rows=rows)

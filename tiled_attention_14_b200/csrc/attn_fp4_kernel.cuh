@@ -22,7 +22,9 @@
 // 512-byte layout the tensor core reads (128 rows x 4 scales: byte 16 (r % 32) + 4 (r / 32)
 // + block), and the MMA thread copies them with tcgen05.cp (32x128b, replicated to the four
 // lane quarters).  P and its scales go through shared memory (FP4 operands come from shared
-// memory), P in the 32-byte swizzle layout, one 32-byte row per query row and key tile.
+// memory), P in the 32-byte swizzle layout, one 32-byte row per query row and key tile.  The
+// row sum of P~ comes from the tensor core too: 16 rows of e2m1 ones below each stage's V^T make
+// the P V product 144 columns wide, column 128 being sum_j P~_j (rescaled with O).
 //
 // Work item: (b, h, 256 query rows) = two 128-row query groups; key tiles of 64 (S is 64
 // columns of tensor memory per group so that both groups' O fit beside it).  Persistent:
@@ -31,7 +33,8 @@
 //   warp  8    producer: Q tiles and scales, then a ring of (128 keys of K, V^T, scales)
 //   warp  9    MMA issuer (one thread); allocates and frees tensor memory
 //   warps 10-11 idle
-// Tensor memory (512 columns): O0 | O1 | S0 | S1 | scale factors.
+// Tensor memory (512 columns): O0 | O1 (144 of 160 each: O and the row sum) | S0 | S1 | scale
+// factors.
 //
 // Every wait is bounded; on time-out the kernel records ATTN_ERR_TIMEOUT, all roles unwind,
 // copies and MMAs in flight are drained (bounded), tensor memory is freed.  Nothing traps.
@@ -87,7 +90,7 @@ __device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t a_desc, uint6
 // all four lane quarters (the scale-factor layout of an M = 128 operand).
 __device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint64_t src_desc) {
 #ifdef ATTN_DEBUG_CHECKS
-  if (!debug_check(tmem_range_ok(taddr, 4))) return;
+  if (!debug_check((taddr >> 16) == 0u && (taddr & 0xFFFFu) + 4u <= 512u)) return;
 #endif
   asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(src_desc) : "memory");
 }
@@ -264,12 +267,14 @@ struct Cfg {
   static constexpr int OFF_Q = 0;                   // Q0, Q1, then their scale atoms
   static constexpr int OFF_QSF = 2 * TILE;
   static constexpr int OFF_KV = 17 * 1024;
-  static constexpr int ST_K = 0, ST_V = TILE, ST_KSF = 2 * TILE, ST_VSF = 2 * TILE + SF;
-  static constexpr int STAGE = 17 * 1024;
+  // K, V^T, then 16 rows of ones below V^T (the row sums as 16 more output columns), scales
+  static constexpr int ST_K = 0, ST_V = TILE, ST_ONES = 2 * TILE, ST_KSF = 2 * TILE + 1024, ST_VSF = ST_KSF + SF;
+  static constexpr int STAGE = 18 * 1024;
   static constexpr int OFF_P = OFF_KV + NS * STAGE;        // P[g][buf]: 128 rows x 32 bytes
   static constexpr int P_TILE = 128 * 32;
   static constexpr int OFF_PSF = OFF_P + 4 * P_TILE;       // P scale atoms [buf] (both groups)
-  static constexpr int OFF_BAR = OFF_PSF + 2 * SF;
+  static constexpr int OFF_ONESF = OFF_PSF + 2 * SF;      // scale atom of the ones rows (all 2^0)
+  static constexpr int OFF_BAR = OFF_ONESF + SF;
   // barriers: QFULL 2, QEMPTY 2, KVFULL NS, KVEMPTY NS, SFULL 2, SFREE 2, PFULL 4, PFREE 4,
   // DRAIN 1.  "P V of tile k of group g is complete" is read from PFREE[g][k & 1]: the
   // softmax waited for that barrier's previous phase before writing P of tile k, so the
@@ -280,13 +285,16 @@ struct Cfg {
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t T_O = 0, T_S = 256, T_SFQ = 384, T_SFP = 392, T_SFK = 408, T_SFV = 424;
+  static constexpr int ON = 144;                          // O columns per group: 128 of O, then the row sum
+  static constexpr uint32_t O_STRIDE = 160;               // group 1's O (32-column aligned)
+  static constexpr uint32_t T_O = 0, T_S = 2 * O_STRIDE, T_SFQ = T_S + 128, T_SFP = T_SFQ + 8, T_SFK = T_SFP + 8,
+                            T_SFV = T_SFK + 4 * NS;            // V^T scales: 8 columns per stage (4 + the ones')
   static constexpr float kTau = 8.f;                 // rescale threshold (octaves)
   static constexpr float kMagic = 12582912.f;        // 1.5 * 2^23: the unit of its last bit is 1
 };
 static_assert(Cfg::OFF_KV >= Cfg::OFF_QSF + 2 * Cfg::SF, "Q region overlaps the ring");
 static_assert(Cfg::SMEM_BYTES <= 227 * 1024, "shared memory");
-static_assert(Cfg::T_SFV + 4 * Cfg::NS <= Cfg::TMEM_COLS, "tensor memory");
+static_assert(Cfg::T_SFV + 8 * Cfg::NS <= Cfg::TMEM_COLS, "tensor memory");
 
 __device__ __forceinline__ void item_of(const Params& p, int w, int& bh, int& qb, int& kvbh) {
   bh = w / p.nqb;
@@ -333,6 +341,13 @@ attn_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     *abort_flag = 0;
     fence_mbar_init();
   }
+  // 16 rows of e2m1 ones (code 2) below each stage's V^T tile, and a scale atom of 2^0: the
+  // P V product then also sums P~ over the keys (output columns 128..143 of each group)
+  for (int i = threadIdx.x; i < C::NS * 256; i += C::THREADS)
+    reinterpret_cast<uint32_t*>(sptr + C::OFF_KV + (i >> 8) * C::STAGE + C::ST_ONES)[i & 255] = 0x22222222u;
+  for (int i = threadIdx.x; i < C::SF / 4; i += C::THREADS)
+    reinterpret_cast<uint32_t*>(sptr + C::OFF_ONESF)[i] = 0x7F7F7F7Fu;
+  fence_proxy_async_smem();
   if (warp == C::MMA_WARP) {
     tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
     tmem_relinquish();
@@ -397,10 +412,12 @@ attn_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   } else if (warp == C::MMA_WARP) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t tO[2] = {tbase + C::T_O, tbase + C::T_O + 128};
+      const uint32_t tO[2] = {tbase + C::T_O, tbase + C::T_O + C::O_STRIDE};
       const uint32_t tS[2] = {tbase + C::T_S, tbase + C::T_S + 64};
       const uint32_t tSFQ[2] = {tbase + C::T_SFQ, tbase + C::T_SFQ + 4};
       auto sfdesc = [&](uint32_t addr) { return sdesc(addr, 16, 128, kLayoutNone); };
+      // the ones rows' scales (2^0) sit in column 4 of every stage's V^T scale columns for good
+      for (int s = 0; s < C::NS; ++s) tmem_cp_sf(tbase + C::T_SFV + 8 * s + 4, sfdesc(sbase + C::OFF_ONESF));
       uint32_t tc = 0, cidx = 0, qcount = 0;
       bool ok = true;
       for (int w = cta; ok && w < p.num_items; w += G) {
@@ -419,7 +436,7 @@ attn_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
               if (!wait_bounded(BAR(C::B_KVFULL + slot), (stage / C::NS) & 1, abort_flag, tmo)) { ok = false; break; }
               tc_fence_after();
               tmem_cp_sf(tbase + C::T_SFK + 4 * slot, sfdesc(st + C::ST_KSF));
-              tmem_cp_sf(tbase + C::T_SFV + 4 * slot, sfdesc(st + C::ST_VSF));
+              tmem_cp_sf(tbase + C::T_SFV + 8 * slot, sfdesc(st + C::ST_VSF));
             }
             const uint32_t t = tc + j;
             for (int g = 0; g < 2; ++g) {
@@ -456,7 +473,7 @@ attn_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             for (int g = 0; g < 2; ++g) {
               const uint64_t a = sdesc(sbase + C::OFF_P + (2 * g + buf) * C::P_TILE, 16, 256, kLayoutSw32);
               const uint64_t b = sdesc(st + C::ST_V + 32 * (jp & 1), 16, 512, kLayoutSw64);
-              mma_mxf4(tO[g], a, b, idesc_mxf4(128, 128, 2 * g, 2 * (jp & 1)), tsfp, tbase + C::T_SFV + 4 * slot,
+              mma_mxf4(tO[g], a, b, idesc_mxf4(128, C::ON, 2 * g, 2 * (jp & 1)), tsfp, tbase + C::T_SFV + 8 * slot,
                        jp > 0 ? 1u : 0u);
               mma_commit(BAR(C::B_PFREE + 2 * g + buf));
             }
@@ -478,7 +495,7 @@ attn_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int rloc = (warp & 3) * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tbase + C::T_S + 64 * g + lane_off;
-    const uint32_t tO = tbase + C::T_O + 128 * g + lane_off;
+    const uint32_t tO = tbase + C::T_O + C::O_STRIDE * g + lane_off;   // O, then the row sum at column 128
     const float c2 = p.c2;
     constexpr float kNegInfF = -__builtin_huge_valf();
     // P row (32 bytes) of this thread in the 32-byte swizzle: chunk c at c ^ bit 2 of the row
@@ -492,7 +509,6 @@ attn_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       item_of(p, w, bh, qb, kvbh);
       const int row = qb * 256 + 128 * g + rloc;
       float m = kNegInfF;     // running reference (an integer, log2 units)
-      float l = 0.f;          // running sum of P~ against 2^m
       for (int j = 0; j < n_sub; ++j) {
         const uint32_t t = tc + j, buf = t & 1;
         if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_SFULL + g), t & 1, abort_flag, tmo))) { ok = false; break; }
@@ -534,7 +550,6 @@ attn_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           if (m != kNegInfF) {
             alpha = exp2i(static_cast<int>(m - mt));
             rescale = true;
-            l *= alpha;
           }
           m = mt;
         }
@@ -551,7 +566,6 @@ attn_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           const bool use = e >= -127;
           const float b8 = use ? (2.5f - 2.f * E[blk]) * 0.125f : kNegInfF;
           sfb |= static_cast<uint32_t>(use ? e + 127 : 0) << (8 * blk);
-          uint32_t acc = 0u;   // per-byte sums of twice the magnitudes (at most 96 per byte)
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             uint32_t byte[4];
@@ -567,10 +581,7 @@ attn_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const uint32_t wv = __byte_perm(__byte_perm(byte[0], byte[1], 0x0040), __byte_perm(byte[2], byte[3], 0x0040),
                                             0x5410);
             pw[4 * blk + q] = wv;
-            // twice the magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6} of the 8 codes, byte by byte
-            acc += __byte_perm(0x03020100u, 0x0C080604u, wv) + __byte_perm(0x03020100u, 0x0C080604u, wv >> 16);
           }
-          if (use) l = fmaf(static_cast<float>(__dp4a(acc, 0x01010101u, 0u)), exp2i(e - 1), l);
         }
         // P and its scales to shared memory (buffer buf is free once PV of tile t-2 is done)
         if (t >= 2 && !__all_sync(0xffffffffu, wait_bounded(BAR(C::B_PFREE + 2 * g + buf), ((t >> 1) - 1) & 1,
@@ -600,6 +611,11 @@ attn_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
             tmem_st_x32_wait<0>(tO + ch * 32, o);
           }
+          uint32_t ls[16];   // the row sum columns
+          tmem_ld_x16_wait(tO + 128, ls);
+#pragma unroll
+          for (int c = 0; c < 16; ++c) ls[c] = __float_as_uint(__uint_as_float(ls[c]) * alpha);
+          tmem_st_x16_wait<0>(tO + 128, ls);
         }
         tc_fence_before();
         if (!(p.fault_skip && g == 1 && t == 0)) mbar_arrive(BAR(C::B_PFULL + 2 * g + buf));
@@ -616,6 +632,9 @@ attn_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         break;
       }
       tc_fence_after();
+      uint32_t ls[16];
+      tmem_ld_x16_wait(tO + 128, ls);
+      const float l = __uint_as_float(ls[0]);   // sum of P~ against 2^m, from the tensor core
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
       __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * p.Sq + row) * 128;
 #pragma unroll
