@@ -275,13 +275,14 @@ struct Cfg {
   static constexpr int OFF_PSF = OFF_P + 4 * P_TILE;       // P scale atoms [buf] (both groups)
   static constexpr int OFF_ONESF = OFF_PSF + 2 * SF;      // scale atom of the ones rows (all 2^0)
   static constexpr int OFF_BAR = OFF_ONESF + SF;
-  // barriers: QFULL 2, QEMPTY 2, KVFULL NS, KVEMPTY NS, SFULL 2, SFREE 2, PFULL 4, PFREE 4,
-  // DRAIN 1.  "P V of tile k of group g is complete" is read from PFREE[g][k & 1]: the
-  // softmax waited for that barrier's previous phase before writing P of tile k, so the
-  // parity it waits for next is never ambiguous.
+  // barriers: QFULL 2, QEMPTY 2, KVFULL NS, KVEMPTY NS, SFULL 2, SFREE 2, PFULL 2, PFREE 2,
+  // DRAIN 1.  PFULL[b] / PFREE[b] serve both groups: P of tile k (buffer k & 1) of both groups
+  // is ready / both P V products of tile k are complete.  "P V of tile k is complete" is read
+  // from PFREE[k & 1]: the softmax waited for that barrier's previous phase before writing P of
+  // tile k, so the parity it waits for next is never ambiguous.
   static constexpr int B_QFULL = 0, B_QEMPTY = 2, B_KVFULL = 4, B_KVEMPTY = 4 + NS, B_SFULL = 4 + 2 * NS,
-                       B_SFREE = B_SFULL + 2, B_PFULL = B_SFREE + 2, B_PFREE = B_PFULL + 4,
-                       B_DRAIN = B_PFREE + 4, NBAR = B_DRAIN + 1;
+                       B_SFREE = B_SFULL + 2, B_PFULL = B_SFREE + 2, B_PFREE = B_PFULL + 2,
+                       B_DRAIN = B_PFREE + 2, NBAR = B_DRAIN + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
@@ -329,8 +330,10 @@ attn_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       mbar_init(BAR(C::B_SFULL + g), 1);
       mbar_init(BAR(C::B_SFREE + g), 128);
       for (int b = 0; b < 2; ++b) {
-        mbar_init(BAR(C::B_PFULL + 2 * g + b), 128);
-        mbar_init(BAR(C::B_PFREE + 2 * g + b), 1);
+        if (g == 0) {
+          mbar_init(BAR(C::B_PFULL + b), 256);   // both groups' P of one tile (one shared scale copy)
+          mbar_init(BAR(C::B_PFREE + b), 1);     // both groups' P V of that tile complete
+        }
       }
     }
     for (int s = 0; s < C::NS; ++s) {
@@ -462,8 +465,7 @@ attn_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const uint32_t st = sbase + C::OFF_KV + slot * C::STAGE;
             // both groups' P scales share one atom (group g in bytes 2g, 2g + 1 of each row):
             // one copy to tensor memory serves both products
-            if (!wait_bounded(BAR(C::B_PFULL + buf), (tp >> 1) & 1, abort_flag, tmo) ||
-                !wait_bounded(BAR(C::B_PFULL + 2 + buf), (tp >> 1) & 1, abort_flag, tmo)) {
+            if (!wait_bounded(BAR(C::B_PFULL + buf), (tp >> 1) & 1, abort_flag, tmo)) {
               ok = false;
               break;
             }
@@ -475,8 +477,8 @@ attn_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
               const uint64_t b = sdesc(st + C::ST_V + 32 * (jp & 1), 16, 512, kLayoutSw64);
               mma_mxf4(tO[g], a, b, idesc_mxf4(128, C::ON, 2 * g, 2 * (jp & 1)), tsfp, tbase + C::T_SFV + 8 * slot,
                        jp > 0 ? 1u : 0u);
-              mma_commit(BAR(C::B_PFREE + 2 * g + buf));
             }
+            mma_commit(BAR(C::B_PFREE + buf));
             if (!ok) break;
             if (jp & 1) mma_commit(BAR(C::B_KVEMPTY + slot));
           }
@@ -584,7 +586,7 @@ attn_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           }
         }
         // P and its scales to shared memory (buffer buf is free once PV of tile t-2 is done)
-        if (t >= 2 && !__all_sync(0xffffffffu, wait_bounded(BAR(C::B_PFREE + 2 * g + buf), ((t >> 1) - 1) & 1,
+        if (t >= 2 && !__all_sync(0xffffffffu, wait_bounded(BAR(C::B_PFREE + buf), ((t >> 1) - 1) & 1,
                                                             abort_flag, tmo))) {
           ok = false;
           break;
@@ -597,7 +599,7 @@ attn_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         fence_proxy_async_smem();
         // rescale O when the reference moved (PV of tile t-1 has completed first)
         if (__any_sync(0xffffffffu, rescale)) {
-          if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_PFREE + 2 * g + ((t - 1) & 1)), ((t - 1) >> 1) & 1,
+          if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_PFREE + ((t - 1) & 1)), ((t - 1) >> 1) & 1,
                                                     abort_flag, tmo))) {
             ok = false;
             break;
@@ -618,7 +620,7 @@ attn_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           tmem_st_x16_wait<0>(tO + 128, ls);
         }
         tc_fence_before();
-        if (!(p.fault_skip && g == 1 && t == 0)) mbar_arrive(BAR(C::B_PFULL + 2 * g + buf));
+        if (!(p.fault_skip && g == 1 && t == 0)) mbar_arrive(BAR(C::B_PFULL + buf));
       }
       if (!__all_sync(0xffffffffu, ok && !*abort_flag)) {
         ok = false;
@@ -626,7 +628,7 @@ attn_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
       // ---- epilogue: O / l -> bf16, LSE
       const uint32_t last = tc + n_sub - 1;
-      if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_PFREE + 2 * g + (last & 1)), (last >> 1) & 1, abort_flag,
+      if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_PFREE + (last & 1)), (last >> 1) & 1, abort_flag,
                                                 tmo))) {
         ok = false;
         break;
