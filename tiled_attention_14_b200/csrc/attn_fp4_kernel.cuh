@@ -275,7 +275,7 @@ struct Cfg {
   static constexpr int OFF_PSF = OFF_P + 4 * P_TILE;       // P scale atoms [buf] (both groups)
   static constexpr int OFF_ONESF = OFF_PSF + 2 * SF;      // scale atom of the ones rows (all 2^0)
   static constexpr int OFF_BAR = OFF_ONESF + SF;
-  // barriers: QFULL 2, QEMPTY 2, KVFULL NS, KVEMPTY NS, SFULL 2, SFREE 2, PFULL 2, PFREE 2,
+  // barriers: QFULL 2, QEMPTY 2, KVFULL NS, KVEMPTY NS, SFULL, SFREE (both groups), PFULL 2, PFREE 2,
   // DRAIN 1.  PFULL[b] / PFREE[b] serve both groups: P of tile k (buffer k & 1) of both groups
   // is ready / both P V products of tile k are complete.  "P V of tile k is complete" is read
   // from PFREE[k & 1]: the softmax waited for that barrier's previous phase before writing P of
@@ -327,8 +327,10 @@ attn_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     for (int g = 0; g < 2; ++g) {
       mbar_init(BAR(C::B_QFULL + g), 1);
       mbar_init(BAR(C::B_QEMPTY + g), 1);
-      mbar_init(BAR(C::B_SFULL + g), 1);
-      mbar_init(BAR(C::B_SFREE + g), 128);
+      if (g == 0) {
+        mbar_init(BAR(C::B_SFULL), 1);     // both groups' S of one tile computed
+        mbar_init(BAR(C::B_SFREE), 256);   // both groups have read their S
+      }
       for (int b = 0; b < 2; ++b) {
         if (g == 0) {
           mbar_init(BAR(C::B_PFULL + b), 256);   // both groups' P of one tile (one shared scale copy)
@@ -442,10 +444,10 @@ attn_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
               tmem_cp_sf(tbase + C::T_SFV + 8 * slot, sfdesc(st + C::ST_VSF));
             }
             const uint32_t t = tc + j;
+            // S0 and S1 are free once both groups' threads have read the previous tile's scores.
+            if (t >= 1 && !wait_bounded(BAR(C::B_SFREE), (t - 1) & 1, abort_flag, tmo)) { ok = false; break; }
+            tc_fence_after();
             for (int g = 0; g < 2; ++g) {
-              // S_g is free once group g's threads have read the previous tile's scores.
-              if (t >= 1 && !wait_bounded(BAR(C::B_SFREE + g), (t - 1) & 1, abort_flag, tmo)) { ok = false; break; }
-              tc_fence_after();
 #pragma unroll
               for (int kk = 0; kk < 2; ++kk) {
                 const uint64_t a = sdesc(sbase + C::OFF_Q + g * C::TILE + 32 * kk, 16, 512, kLayoutSw64);
@@ -453,9 +455,9 @@ attn_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 mma_mxf4(tS[g], a, b, idesc_mxf4(128, 64, 2 * kk, 2 * kk), tSFQ[g],
                          tbase + C::T_SFK + 4 * slot + 2 * (j & 1), kk > 0);
               }
-              mma_commit(BAR(C::B_SFULL + g));
               if (j == n_sub - 1) mma_commit(BAR(C::B_QEMPTY + g));   // last read of Q_g
             }
+            mma_commit(BAR(C::B_SFULL));
             if (!ok) break;
           }
           if (j >= 1) {
@@ -513,12 +515,12 @@ attn_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       float m = kNegInfF;     // running reference (an integer, log2 units)
       for (int j = 0; j < n_sub; ++j) {
         const uint32_t t = tc + j, buf = t & 1;
-        if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_SFULL + g), t & 1, abort_flag, tmo))) { ok = false; break; }
+        if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_SFULL), t & 1, abort_flag, tmo))) { ok = false; break; }
         tc_fence_after();
         uint32_t s[64];
         tmem_ld_x64_wait(tS, s);
         tc_fence_before();
-        mbar_arrive(BAR(C::B_SFREE + g));
+        mbar_arrive(BAR(C::B_SFREE));
         // keys past the end of the sequence take no part
         const int nvalid = p.Sk - 64 * j;
         if (nvalid < 64) {
