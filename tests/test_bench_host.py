@@ -97,3 +97,17 @@ def test_profiled_traffic_is_gated_by_the_kernel_source_hash(tmp_path, monkeypat
     assert bench.profiled_traffic("causal") == 123.0
     (csrc / "attn_fwd_kernel.cuh").write_text("// kernel v2\n")        # the kernel changed since
     assert bench.profiled_traffic("causal") is None
+
+
+def test_fp4_workload_accounting():
+    """FP4 long: the algorithmic FLOPs of the BF16 long shape, compulsory bytes of the e2m1 codes
+    (V padded to 128 keys), the scale atoms, O and LSE, and the FP4 peak as FP8 x 2."""
+    w = bench.WORKLOADS["fp4_long"]
+    assert w.fp4 and not w.fp8 and w.mask_kind == 0
+    assert bench.algorithmic_flops(w) == bench.algorithmic_flops(bench.WORKLOADS["long"])
+    nq = nk = 32768 // 128
+    expect = 32 * 32768 * 64 + 2 * 32 * nk * 128 * 64 + 32 * (nq + 2 * nk) * 512 + 32 * 32768 * (128 * 2 + 4)
+    assert bench.compulsory_bytes(w) == expect
+    assert bench.dtype_of(w) == "e2m1" and bench.peak_key(w) == "fp4"
+    peaks = bench.measured_peaks()
+    assert peaks["fp4"] == 2 * peaks["fp8"]

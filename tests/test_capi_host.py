@@ -118,6 +118,20 @@ def test_binding_rejects_host_tensors_and_bad_outputs():
         ta.attn_fwd(meta, meta, meta)
     with pytest.raises(ValueError):
         ta.attn_quantize_e4m3(torch.zeros(1, 1, 128, 128))
+    with pytest.raises(ValueError):
+        ta.attn_quantize_mxfp4(q)                    # host tensor
+    u8 = torch.zeros(1, 1, 128, 64, dtype=torch.uint8)
+    with pytest.raises(ValueError):
+        ta.attn_fwd_fp4(u8, u8, u8, u8, u8, u8, 128)    # host tensors
+
+
+def test_mxfp4_shapes():
+    """Storage shapes of the MXFP4 tensors: 64 bytes per row of 128 elements; V transposed with
+    its keys padded to 128; one 512-byte scale atom per 128 rows (or keys)."""
+    import tiled_attention_14_b200 as ta
+    assert ta.mxfp4_shapes(2, 3, 300) == ((2, 3, 300, 64), (2, 3, 3, 512))
+    assert ta.mxfp4_shapes(2, 3, 300, transpose=True) == ((2, 3, 128, 192), (2, 3, 3, 512))
+    assert ta.mxfp4_shapes(1, 1, 1, transpose=True) == ((1, 1, 128, 64), (1, 1, 1, 512))
 
 
 ABL_SIGNATURES = {
