@@ -17,6 +17,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import math
 import os
@@ -202,11 +203,19 @@ FWD_SOURCES = ("attn_fwd_kernel.cuh", "ptx.cuh", "tmem_moves.cuh", "attn_api.cu"
                "attn_fp4_api.inc")
 
 
+def code_only(text: str) -> str:
+    """The source without its comments and blank lines (no source here puts a comment marker
+    inside a string literal), so that a comment edit does not invalidate a capture."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lines = (re.sub(r"//.*", "", line).rstrip() for line in text.splitlines())
+    return "\n".join(line for line in lines if line.strip())
+
+
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "tiled_attention_14_b200", "csrc")
     for f in FWD_SOURCES:
-        h.update(open(os.path.join(csrc, f), "rb").read())
+        h.update(code_only(open(os.path.join(csrc, f), encoding="utf-8").read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -80,12 +80,13 @@ def test_committed_traffic_files_are_well_formed():
 
 
 def test_profiled_traffic_is_gated_by_the_kernel_source_hash(tmp_path, monkeypatch):
-    """A traffic figure is reported only while the kernel sources match the capture."""
+    """A traffic figure is reported only while the kernel sources' code (comments aside) matches
+    the capture."""
     csrc = tmp_path / "tiled_attention_14_b200" / "csrc"
     csrc.mkdir(parents=True)
     for f in bench.FWD_SOURCES:
         (csrc / f).write_text("// source\n")
-    (csrc / "attn_fwd_kernel.cuh").write_text("// kernel v1\n")
+    (csrc / "attn_fwd_kernel.cuh").write_text("// kernel\nint v = 1;\n")
     (tmp_path / "profiles").mkdir()
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     h = bench.kernel_source_hash()
@@ -95,7 +96,9 @@ def test_profiled_traffic_is_gated_by_the_kernel_source_hash(tmp_path, monkeypat
     assert bench.profiled_traffic("long") is None              # no capture for this workload
     (csrc / "attn_bwd_kernel.cuh").write_text("// another kernel\n")   # not part of the forward
     assert bench.profiled_traffic("causal") == 123.0
-    (csrc / "attn_fwd_kernel.cuh").write_text("// kernel v2\n")        # the kernel changed since
+    (csrc / "attn_fwd_kernel.cuh").write_text("/* kernel */ // edited comment\n\nint v = 1;  // here\n")
+    assert bench.profiled_traffic("causal") == 123.0          # comments and blank lines only
+    (csrc / "attn_fwd_kernel.cuh").write_text("// kernel\nint v = 2;\n")   # the kernel changed since
     assert bench.profiled_traffic("causal") is None
 
 

@@ -17,7 +17,8 @@
 //   O = sum P~ V / sum P~, LSE = ln(sum P~), with P~ the magnitudes the tensor core multiplied.
 //
 // Both products run as tcgen05.mma kind::mxf4 (block32, E8M0 scales): S = Q K^T with
-// M = 128, N = 64, K = 128 (two instructions), O += P V with M = 128, N = 128, K = 64 (one).
+// M = 128, N = 64, K = 128 (two instructions), O += P V with M = 128, N = 144 (128 of O and 16
+// of row sums, below), K = 64 (one).
 // Scale factors live in tensor memory; the producer brings them into shared memory in the
 // 512-byte layout the tensor core reads (128 rows x 4 scales: byte 16 (r % 32) + 4 (r / 32)
 // + block), and the MMA thread copies them with tcgen05.cp (32x128b, replicated to the four
