@@ -114,6 +114,14 @@ def test_fp4_forward_peaked_and_flat_rows(mul):
     _check(q, k, v)
 
 
+@pytest.mark.parametrize("scale", [0.02, 0.3])
+def test_fp4_forward_other_scales(scale):
+    """A softmax scale other than 1/sqrt(D): the kernel's score-to-code constant and the
+    oracle's both follow the scale argument (small: nearly flat rows; large: peaked rows)."""
+    q, k, v = make_qkv(1, 2, 300, 520, 128, seed=15)
+    _check(q, k, v, scale=scale)
+
+
 def test_fp4_forward_full_size_sampled_rows():
     """The non-causal inference shape (B1 H32 S32768 D128), sampled rows of three heads."""
     q, k, v = make_qkv(1, 32, 32768, 32768, 128, seed=0)
