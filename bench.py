@@ -197,10 +197,12 @@ class ClockSampler:
                 "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
-# The sources that make up the forward attention kernels (BF16/FP8 and FP4) and their launch
-# (the backward, quantiser and tile-map sources do not change them).
-FWD_SOURCES = ("attn_fwd_kernel.cuh", "ptx.cuh", "tmem_moves.cuh", "attn_api.cu", "attn_fp4_kernel.cuh",
-               "attn_fp4_api.inc")
+# The sources that make up each forward attention kernel family and its launch: BF16/FP8
+# (attn_fwd_kernel) and FP4 (attn_fp4_kernel, which also uses the BF16 kernel's helpers).  The
+# backward, quantiser and tile-map sources do not change them.
+BF16_SOURCES = ("attn_fwd_kernel.cuh", "ptx.cuh", "tmem_moves.cuh", "attn_api.cu")
+FP4_SOURCES = BF16_SOURCES + ("attn_fp4_kernel.cuh", "attn_fp4_api.inc")
+FWD_SOURCES = FP4_SOURCES
 
 
 def code_only(text: str) -> str:
@@ -211,10 +213,11 @@ def code_only(text: str) -> str:
     return "\n".join(line for line in lines if line.strip())
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(family: str = "bf16") -> str:
+    """Hash of the code (comments and blank lines removed) of one kernel family's sources."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "tiled_attention_14_b200", "csrc")
-    for f in FWD_SOURCES:
+    for f in (FP4_SOURCES if family == "fp4" else BF16_SOURCES):
         h.update(code_only(open(os.path.join(csrc, f), encoding="utf-8").read()).encode())
     return h.hexdigest()[:16]
 
@@ -226,7 +229,8 @@ def profiled_traffic(workload: str):
     if not os.path.exists(p):
         return None
     d = json.load(open(p))
-    if d.get("kernel_source_hash") != kernel_source_hash():
+    w = WORKLOADS.get(workload)
+    if d.get("kernel_source_hash") != kernel_source_hash("fp4" if (w is not None and w.fp4) else "bf16"):
         return None
     return d.get("dram_bytes_per_launch")
 

@@ -102,6 +102,26 @@ def test_profiled_traffic_is_gated_by_the_kernel_source_hash(tmp_path, monkeypat
     assert bench.profiled_traffic("causal") is None
 
 
+def test_profiled_traffic_hash_is_per_kernel_family(tmp_path, monkeypatch):
+    """An FP4 kernel change invalidates the FP4 capture only; a change to the sources both
+    families share invalidates both."""
+    csrc = tmp_path / "tiled_attention_14_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    for f in bench.FP4_SOURCES:
+        (csrc / f).write_text(f"int {f.split('.')[0]} = 1;\n")
+    (tmp_path / "profiles").mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    for wl, fam in (("causal", "bf16"), ("fp4_long", "fp4")):
+        rec = {"workload": wl, "kernel_source_hash": bench.kernel_source_hash(fam), "dram_bytes_per_launch": 7.0}
+        (tmp_path / "profiles" / f"traffic_{wl}.json").write_text(json.dumps(rec))
+    assert bench.kernel_source_hash("bf16") != bench.kernel_source_hash("fp4")
+    assert bench.profiled_traffic("causal") == 7.0 and bench.profiled_traffic("fp4_long") == 7.0
+    (csrc / "attn_fp4_kernel.cuh").write_text("int attn_fp4_kernel = 2;\n")
+    assert bench.profiled_traffic("causal") == 7.0 and bench.profiled_traffic("fp4_long") is None
+    (csrc / "ptx.cuh").write_text("int ptx = 2;\n")
+    assert bench.profiled_traffic("causal") is None
+
+
 def test_fp4_workload_accounting():
     """FP4 long: the algorithmic FLOPs of the BF16 long shape, compulsory bytes of the e2m1 codes
     (V padded to 128 keys), the scale atoms, O and LSE, and the FP4 peak as FP8 x 2."""

@@ -330,11 +330,11 @@ attn_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       mbar_init(BAR(C::B_QEMPTY + g), 1);
       if (g == 0) {
         mbar_init(BAR(C::B_SFULL), 1);     // both groups' S of one tile computed
-        mbar_init(BAR(C::B_SFREE), 256);   // both groups have read their S
+        mbar_init(BAR(C::B_SFREE), 8);     // both groups have read their S (one arrival per softmax warp)
       }
       for (int b = 0; b < 2; ++b) {
         if (g == 0) {
-          mbar_init(BAR(C::B_PFULL + b), 256);   // both groups' P of one tile (one shared scale copy)
+          mbar_init(BAR(C::B_PFULL + b), 8);     // both groups' P of one tile (one arrival per softmax warp)
           mbar_init(BAR(C::B_PFREE + b), 1);     // both groups' P V of that tile complete
         }
       }
@@ -521,7 +521,8 @@ attn_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         uint32_t s[64];
         tmem_ld_x64_wait(tS, s);
         tc_fence_before();
-        mbar_arrive(BAR(C::B_SFREE));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(C::B_SFREE));
         // keys past the end of the sequence take no part
         const int nvalid = p.Sk - 64 * j;
         if (nvalid < 64) {
@@ -623,7 +624,9 @@ attn_fp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           tmem_st_x16_wait<0>(tO + 128, ls);
         }
         tc_fence_before();
-        if (!(p.fault_skip && g == 1 && t == 0)) mbar_arrive(BAR(C::B_PFULL + buf));
+        // one arrival per warp: the warp's stores and fences above come first
+        __syncwarp();
+        if (lane == 0 && !(p.fault_skip && g == 1 && t == 0)) mbar_arrive(BAR(C::B_PFULL + buf));
       }
       if (!__all_sync(0xffffffffu, ok && !*abort_flag)) {
         ok = false;
